@@ -1,0 +1,117 @@
+"""Seeded synthetic workloads shared by the tests, the bench and the oracle runs.
+
+This module holds no attention arithmetic: it only names the benchmark shapes and
+draws the random tensors.  Both the CUDA path and the fp64 CPU oracle are fed from
+here, so the two sides see bit-identical inputs.
+
+Workload geometry follows the attention-kernel sweep described in "FlashAttention-2を読む"
+(section "約2倍という数値の対象を確認する"): sequence length 512 .. 16k, head dim 64 / 128,
+causal on and off, the total number of tokens per batch fixed at 16k.  The hidden size
+H*d = 2048 and the long-context / fp32-tiny cases are this library's own choices.
+
+Recipe: every value is an iid standard normal drawn in fp32 by a CPU
+``torch.Generator`` seeded with ``seed``, in the order q, k, v, dO, each of shape
+[B, N, H, d] (the (batch, seq, heads, head_dim) layout used by ``flash_attn_func``);
+bf16 workloads then round to bf16 (round to nearest even).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Dict, List, Optional
+
+import torch
+
+TOTAL_TOKENS = 16384
+SWEEP_N = [512, 1024, 2048, 4096, 8192, 16384]
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One attention problem: shapes, precision, masking and seed."""
+
+    name: str
+    B: int
+    N: int
+    H: int
+    d: int
+    causal: bool
+    dtype: str  # "bf16" or "f32"
+    backward: bool
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / (self.d ** 0.5)
+
+    @property
+    def tokens(self) -> int:
+        return self.B * self.N
+
+    def fwd_flops(self) -> float:
+        """4*B*H*N^2*d, halved under the causal mask (the usual attention FLOP count)."""
+        f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        return f / 2 if self.causal else f
+
+    def bwd_flops(self) -> float:
+        return 2.5 * self.fwd_flops()
+
+    def label(self) -> str:
+        return (f"{self.name}:B{self.B}xN{self.N}xH{self.H}xd{self.d}"
+                f"{'-causal' if self.causal else ''}-{self.dtype}")
+
+
+def tiny_f32(causal: bool) -> Workload:
+    return Workload("tiny_f32", 1, 128, 2, 64, causal, "f32", False, 1000)
+
+
+def fwd_sweep(d: int, N: int, causal: bool) -> Workload:
+    H = 2048 // d
+    return Workload(f"fwd_d{d}", TOTAL_TOKENS // N, N, H, d, causal, "bf16", False,
+                    1001 if d == 64 else 1002)
+
+
+def fwdbwd(N: int) -> Workload:
+    return Workload("fwdbwd_d128", TOTAL_TOKENS // N, N, 16, 128, True, "bf16", True, 1003)
+
+
+def long_context() -> Workload:
+    return Workload("long_64k", 1, 65536, 16, 128, True, "bf16", True, 1004)
+
+
+def all_workloads() -> List[Workload]:
+    out = [tiny_f32(False), tiny_f32(True)]
+    for d in (64, 128):
+        for N in SWEEP_N:
+            for c in (False, True):
+                out.append(fwd_sweep(d, N, c))
+    for N in SWEEP_N[1:]:
+        out.append(fwdbwd(N))
+    out.append(long_context())
+    return out
+
+
+def draw(B: int, N: int, H: int, d: int, seed: int, dtype: str = "bf16",
+         with_grad: bool = False) -> Dict[str, torch.Tensor]:
+    """Draw q, k, v (and dO) on the CPU.  Returns contiguous [B, N, H, d] tensors."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    names = ["q", "k", "v"] + (["dO"] if with_grad else [])
+    out = {}
+    for nm in names:
+        t = torch.randn((B, N, H, d), generator=g, dtype=torch.float32)
+        if dtype == "bf16":
+            t = t.to(torch.bfloat16)
+        elif dtype != "f32":
+            raise ValueError(f"unknown dtype {dtype}")
+        out[nm] = t.contiguous()
+    return out
+
+
+def draw_workload(w: Workload, with_grad: Optional[bool] = None) -> Dict[str, torch.Tensor]:
+    return draw(w.B, w.N, w.H, w.d, w.seed, w.dtype,
+                w.backward if with_grad is None else with_grad)
+
+
+def to_f64(t: torch.Tensor):
+    """Exact upcast of a bf16/fp32 tensor to a float64 numpy array."""
+    return t.to(torch.float64).numpy()
