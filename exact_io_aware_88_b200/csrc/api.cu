@@ -1,0 +1,253 @@
+// api.cu -- the C ABI (include/fa.h, include/fa_debug.h): argument validation, TMA
+// descriptor encoding, device status word, and dispatch to the kernels.  No entry point
+// allocates device memory, synchronises (except fa_read_device_status) or throws.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "fa.h"
+#include "fa_debug.h"
+#include "launch.h"
+
+namespace {
+
+// Library-owned device status word (FA_OK / FA_ERR_TIMEOUT); one per device context.
+__device__ int g_fa_status = 0;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  bool sm100 = false;
+  int num_sms = 0;
+  int* status = nullptr;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Looks up (once per device) the SM count, whether it is an sm_100 part and the device
+// address of the status word; also resolves cuTensorMapEncodeTiled through the runtime so
+// that the library needs no link-time dependency on libcuda.
+int device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fa_status) != cudaSuccess) return FA_ERR_CUDA;
+    if (!g_encode) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return FA_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    d.sm100 = (major == 10 && minor == 0);
+    d.num_sms = sms;
+    d.status = static_cast<int*>(p);
+    d.ready = true;
+  }
+  *out = d;
+  return d.sm100 ? FA_OK : FA_ERR_UNSUPPORTED;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape checks shared by the bf16 entry points.  Returns FA_OK or an error code.
+int check_shape(int B, int H, int N, int d, float scale) {
+  if (B < 1 || H < 1 || N < 1 || !isfinite(scale)) return FA_ERR_INVALID_ARG;
+  const long double elems = static_cast<long double>(B) * N * H * d;
+  if (elems > 9.0e15L) return FA_ERR_INVALID_ARG;
+  const long long tiles = static_cast<long long>(B) * H * ((N + 127) / 128);
+  if (tiles > 0x7fffffffLL || N > 0x7fffff80) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+// 4-D view [B][N][H][d] (innermost first: d, H, N, B) of a bf16 tensor, tiled in boxes of
+// 64 d-elements (128 bytes, the 128-byte swizzle span) x 1 head x 128 rows x 1 batch.
+int encode_bnhd(CUtensorMap* m, const void* ptr, int B, int N, int H, int d) {
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(H) * d * 2,
+                                 static_cast<cuuint64_t>(N) * H * d * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+int from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return FA_OK;
+  if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
+  return FA_ERR_CUDA;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported (head dim or device)";
+    case FA_ERR_MISALIGNED: return "misaligned pointer";
+    case FA_ERR_WORKSPACE: return "workspace missing or too small";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int fa_version(void) { return 100; }
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+           int d, int causal, float scale, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  int rc = check_shape(B, H, N, d, scale);
+  if (rc) return rc;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4))
+    return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  fa::FwdArgs a;
+  if ((rc = encode_bnhd(&a.tm_q, q, B, N, H, d)) || (rc = encode_bnhd(&a.tm_k, k, B, N, H, d)) ||
+      (rc = encode_bnhd(&a.tm_v, v, B, N, H, d)))
+    return rc;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.d = d;
+  a.causal = causal ? 1 : 0;
+  a.scale = scale;
+  a.status = di.status;
+  a.num_sms = di.num_sms;
+  return from_cuda(fa::launch_fwd_sm100(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d, 1.0f) != FA_OK || d < 1) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  return round_up(rows * d * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal,
+           float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  int rc = check_shape(B, H, N, d, scale);
+  if (rc) return rc;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dO, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 16))
+    return FA_ERR_MISALIGNED;
+  const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  fa::BwdArgs a;
+  if ((rc = encode_bnhd(&a.tm_q, q, B, N, H, d)) || (rc = encode_bnhd(&a.tm_k, k, B, N, H, d)) ||
+      (rc = encode_bnhd(&a.tm_v, v, B, N, H, d)) || (rc = encode_bnhd(&a.tm_do, dO, B, N, H, d)))
+    return rc;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  a.o = o;
+  a.dO = dO;
+  a.lse = lse;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dq_acc = static_cast<float*>(workspace);
+  a.delta = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                     round_up(rows * d * sizeof(float), 256));
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.d = d;
+  a.causal = causal ? 1 : 0;
+  a.scale = scale;
+  a.status = di.status;
+  a.num_sms = di.num_sms;
+  return from_cuda(fa::launch_bwd_sm100(a, static_cast<cudaStream_t>(stream)));
+}
+
+int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H,
+               int N, int d, int causal, float scale, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || !isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d < 1 || d > 128 || (d % 4) != 0) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > 65535 || static_cast<long double>(B) * N * H * d > 9.0e15L)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4))
+    return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  return from_cuda(fa::launch_fwd_f32(q, k, v, o, lse, B, H, N, d, causal ? 1 : 0, scale,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+int fa_read_device_status(int* status_out, void* stream) {
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  int word = 0;
+  const int zero = 0;
+  if (cudaMemcpy(&word, di.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(di.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (status_out) *status_out = word;
+  return word;
+}
+
+int fa_debug_umma_tile(const void* a, const void* b, float* c, int n, int k, int mode,
+                       void* stream) {
+  if (!a || !b || !c) return FA_ERR_INVALID_ARG;
+  if ((n != 64 && n != 128) || (k != 64 && k != 128) || mode < 0 || mode > 2)
+    return FA_ERR_UNSUPPORTED;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(c, 16)) return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  return from_cuda(
+      fa::launch_debug_umma(a, b, c, n, k, mode, di.status, static_cast<cudaStream_t>(stream)));
+}
+
+int fa_debug_wait_timeout(long long timeout_ns, void* stream) {
+  if (timeout_ns < 1000 || timeout_ns > 10000000000LL) return FA_ERR_INVALID_ARG;
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  return from_cuda(fa::launch_debug_wait_timeout(static_cast<uint64_t>(timeout_ns), di.status,
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

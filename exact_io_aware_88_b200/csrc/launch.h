@@ -1,0 +1,49 @@
+// launch.h -- internal interface between the C ABI layer (api.cu) and the kernel
+// translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa {
+
+// Default upper bound on any single in-kernel wait (nanoseconds).  A healthy kernel
+// never waits anywhere near this long; hitting it means a pipeline stalled.
+constexpr uint64_t kDefaultWaitTimeoutNs = 4000000000ull;
+
+struct FwdArgs {
+  CUtensorMap tm_q, tm_k, tm_v;  // 4-D maps over [B][N][H][d] bf16, box {64,1,128,1}
+  void* o;
+  float* lse;
+  int B, H, N, d, causal;
+  float scale;
+  int* status;
+  int num_sms;
+};
+
+struct BwdArgs {
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;  // 4-D maps, box {64,1,128,1}
+  const void* o;
+  const void* dO;
+  const float* lse;
+  void *dq, *dk, *dv;
+  float* dq_acc;  // [B][H][N][d] fp32 workspace
+  float* delta;   // [B][H][N] fp32 workspace
+  int B, H, N, d, causal;
+  float scale;
+  int* status;
+  int num_sms;
+};
+
+cudaError_t launch_fwd_sm100(const FwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_sm100(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
+                           int B, int H, int N, int d, int causal, float scale, cudaStream_t s);
+
+// Debug / self-test kernels (fa_debug.h).
+cudaError_t launch_debug_umma(const void* a, const void* b, float* c, int n, int k, int mode,
+                              int* status, cudaStream_t s);
+cudaError_t launch_debug_wait_timeout(uint64_t timeout_ns, int* status, cudaStream_t s);
+
+}  // namespace fa

@@ -1,0 +1,178 @@
+"""ctypes binding of libfa.so (include/fa.h, include/fa_debug.h).
+
+Argument marshalling only: every step of the attention path runs in the library's CUDA
+kernels.  There is no CPU fallback; if libfa.so is missing or cannot be loaded, importing
+this module raises.
+
+The ``fa_*`` functions mirror the C entry points one to one and accept either raw device
+addresses (ints) or torch tensors (their ``data_ptr()`` is passed).  ``attention_forward``
+and ``attention_backward`` are conveniences that allocate outputs with torch and call them.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_MISALIGNED = 3
+FA_ERR_WORKSPACE = 4
+FA_ERR_CUDA = 5
+FA_ERR_TIMEOUT = 6
+
+
+class FAError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {code} ({status_string(code)})")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it first "
+                          "(python -c 'import __graft_entry__ as g; g.build()')")
+    return ctypes.CDLL(LIB_PATH)
+
+
+_lib = _load()
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+_lib.fa_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
+_lib.fa_fwd.restype = _I
+_lib.fa_bwd_workspace_bytes.argtypes = [_I, _I, _I, _I]
+_lib.fa_bwd_workspace_bytes.restype = _SZ
+_lib.fa_bwd.argtypes = [_P] * 9 + [_I, _I, _I, _I, _I, _F, _P, _SZ, _P]
+_lib.fa_bwd.restype = _I
+_lib.fa_fwd_f32.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
+_lib.fa_fwd_f32.restype = _I
+_lib.fa_read_device_status.argtypes = [ctypes.POINTER(_I), _P]
+_lib.fa_read_device_status.restype = _I
+_lib.fa_status_string.argtypes = [_I]
+_lib.fa_status_string.restype = ctypes.c_char_p
+_lib.fa_version.argtypes = []
+_lib.fa_version.restype = _I
+_lib.fa_debug_umma_tile.argtypes = [_P, _P, _P, _I, _I, _I, _P]
+_lib.fa_debug_umma_tile.restype = _I
+_lib.fa_debug_wait_timeout.argtypes = [ctypes.c_longlong, _P]
+_lib.fa_debug_wait_timeout.restype = _I
+
+# Every symbol the C headers declare, for the ABI self-check.
+EXPORTED = ["fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_fwd_f32", "fa_read_device_status",
+            "fa_status_string", "fa_version", "fa_debug_umma_tile", "fa_debug_wait_timeout"]
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, torch.Tensor):
+        return x.data_ptr()
+    return int(x)
+
+
+def _stream(s) -> Optional[int]:
+    if s is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(s, torch.cuda.Stream):
+        return s.cuda_stream
+    return int(s)
+
+
+def status_string(code: int) -> str:
+    return _lib.fa_status_string(int(code)).decode()
+
+
+def version() -> int:
+    return _lib.fa_version()
+
+
+def fa_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, stream=None) -> int:
+    return _lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, int(causal),
+                       float(scale), _stream(stream))
+
+
+def fa_bwd_workspace_bytes(B, H, N, d) -> int:
+    return _lib.fa_bwd_workspace_bytes(B, H, N, d)
+
+
+def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, workspace,
+           workspace_bytes, stream=None) -> int:
+    return _lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                       _ptr(dk), _ptr(dv), B, H, N, d, int(causal), float(scale),
+                       _ptr(workspace), int(workspace_bytes), _stream(stream))
+
+
+def fa_fwd_f32(q, k, v, o, lse, B, H, N, d, causal, scale, stream=None) -> int:
+    return _lib.fa_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                           int(causal), float(scale), _stream(stream))
+
+
+def fa_read_device_status(stream=None) -> int:
+    word = _I(0)
+    return _lib.fa_read_device_status(ctypes.byref(word), _stream(stream))
+
+
+def fa_debug_umma_tile(a, b, c, n, k, mode, stream=None) -> int:
+    return _lib.fa_debug_umma_tile(_ptr(a), _ptr(b), _ptr(c), n, k, mode, _stream(stream))
+
+
+def fa_debug_wait_timeout(timeout_ns, stream=None) -> int:
+    return _lib.fa_debug_wait_timeout(int(timeout_ns), _stream(stream))
+
+
+# ------------------------------------------------------------------ tensor conveniences
+
+def _check(fn: str, rc: int):
+    if rc != FA_OK:
+        raise FAError(fn, rc)
+
+
+def _shape(q: torch.Tensor):
+    if q.dim() != 4:
+        raise ValueError("expected [B, N, H, d] tensors")
+    return q.shape
+
+
+def attention_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+                      scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                      lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """O, LSE for [B, N, H, d] CUDA tensors (bf16 -> fa_fwd, fp32 -> fa_fwd_f32)."""
+    B, N, H, d = _shape(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    for t in (q, k, v):
+        if not (t.is_cuda and t.is_contiguous() and t.shape == q.shape and t.dtype == q.dtype):
+            raise ValueError("q, k, v must be contiguous CUDA tensors of one shape and dtype")
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    if q.dtype == torch.bfloat16:
+        _check("fa_fwd", fa_fwd(q, k, v, o, l, B, H, N, d, causal, scale))
+    elif q.dtype == torch.float32:
+        _check("fa_fwd_f32", fa_fwd_f32(q, k, v, o, l, B, H, N, d, causal, scale))
+    else:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    return o, l
+
+
+def attention_backward(q, k, v, o, lse, dO, causal: bool = False, scale: Optional[float] = None,
+                       workspace: Optional[torch.Tensor] = None):
+    """dQ, dK, dV for bf16 [B, N, H, d] CUDA tensors."""
+    B, N, H, d = _shape(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    nbytes = fa_bwd_workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(nbytes, device=q.device, dtype=torch.uint8)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    _check("fa_bwd", fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale,
+                            workspace, workspace.numel() * workspace.element_size()))
+    return dq, dk, dv

@@ -1,0 +1,101 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library (libfa.so).
+ *
+ * What is computed.  Exact scaled-dot-product attention
+ *     O = softmax(scale * Q K^T [+ causal mask]) V
+ * as written in "Flash Attention 2で打破するローカルLLMの「メモリの壁」" (section
+ * 標準的なAttention機構のメモリ挙動, the Attention(Q,K,V) formula), evaluated the IO-aware
+ * way the same page describes (section タイリング（Tiling）と再計算（Recomputation）の仕組み):
+ * Q, K and V move through on-chip memory in tiles, a running max / sum per row keeps the
+ * softmax globally normalised ("FlashAttention-2を読む", section タイル分割でも全体の
+ * 正規化を保つ), and only O and the per-row logsumexp reach device memory.  The backward
+ * pass recomputes S and P from the logsumexp instead of storing them.
+ *
+ * Conventions shared by every entry point:
+ *  - Tensor layout: q, k, v, o, dO, dq, dk, dv are contiguous [B][N][H][d] arrays (the
+ *    (batch, seq, heads, head_dim) order of flash_attn_func on the same page, section
+ *    カスタムモデルへの組み込み).  lse is a contiguous [B][H][N] fp32 array.
+ *  - lse[b][h][i] = ln sum_j exp(scale * q_i . k_j) over the keys visible to query i
+ *    (natural log, scale included).
+ *  - Causal mask: key j is visible to query i iff j <= i.  Q and K have the same length N.
+ *  - scale is passed explicitly (1/sqrt(d) gives the textbook softmax).
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  No entry point
+ *    allocates, frees or synchronises (except fa_read_device_status); work is enqueued on
+ *    `stream` (a cudaStream_t passed as void*, NULL = legacy default stream).
+ *  - Alignment: every bf16 / fp32 tensor pointer must be 16-byte aligned (the TMA and
+ *    vector-store rule) except fa_fwd / fa_fwd_f32's lse (4 bytes); else FA_ERR_MISALIGNED.
+ *  - Return value: FA_OK (0) on success, else an fa_status code.  On any non-zero return
+ *    nothing was launched and no output was touched.  No C++ exception crosses the ABI.
+ *  - Device-side failures (a bounded wait inside a kernel that ran out) do not trap the
+ *    GPU: the kernel records FA_ERR_TIMEOUT in a library-owned device status word, tears
+ *    its CTA down cleanly and returns; read it with fa_read_device_status().
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* B, H or N < 1, a null pointer, non-finite scale, size overflow */
+  FA_ERR_UNSUPPORTED = 2, /* head dim not supported by this entry point / no sm_100 device */
+  FA_ERR_MISALIGNED = 3,  /* a pointer not 16-byte aligned                                */
+  FA_ERR_WORKSPACE = 4,   /* workspace null or smaller than fa_bwd_workspace_bytes()      */
+  FA_ERR_CUDA = 5,        /* a CUDA runtime / driver call failed (launch, attribute, ...) */
+  FA_ERR_TIMEOUT = 6      /* a device-side bounded wait expired (read via status word)    */
+} fa_status;
+
+/* Forward pass, bf16 in / bf16 out, fp32 accumulation and statistics.
+ *   q, k, v : [B][N][H][d] bf16 (read)        o   : [B][N][H][d] bf16 (written)
+ *   lse     : [B][H][N] fp32 (written), 4-byte aligned
+ *   d must be 64 or 128 (else FA_ERR_UNSUPPORTED).
+ * Kernel: persistent, warp-specialised tcgen05 (TMEM accumulators, TMA K/V ring). */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/* Bytes of device workspace fa_bwd needs for this problem: an fp32 dQ accumulator
+ * (B*H*N*d floats) and the fp32 row statistic D (B*H*N floats), each 256-byte aligned.
+ * Returns 0 if the arguments are invalid. */
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/* Backward pass.  Inputs are the forward's q, k, v, its outputs o and lse, and the
+ * upstream gradient dO (all [B][N][H][d] bf16 except lse, which must be 16-byte
+ * aligned here).  Writes dq, dk, dv
+ * ([B][N][H][d] bf16).  `workspace` is caller-owned device memory of at least
+ * fa_bwd_workspace_bytes(B, H, N, d) bytes; its contents on entry are ignored and on
+ * return are unspecified.  d must be 64 or 128.
+ * Steps: D = rowsum(dO o O) with dQ-accumulator clearing; per key/value tile, recompute
+ * S^T and P^T from lse, dP^T = V dO^T, dS^T = P^T o (dP^T - D); dV += P^T dO and
+ * dK += dS^T Q accumulate in TMEM; dQ += dS K is reduced in fp32 into the workspace
+ * and converted to bf16 (times scale) by a final pass. */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv,
+           int B, int H, int N, int d, int causal, float scale,
+           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Forward pass in fp32 on the CUDA cores (no tensor cores, no TF32), for fp32 inputs.
+ *   q, k, v, o : [B][N][H][d] fp32; lse : [B][H][N] fp32.  1 <= d <= 128, d % 4 == 0. */
+int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
+               int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/* Synchronises `stream`, then returns and clears the library's device status word
+ * (FA_OK or FA_ERR_TIMEOUT).  If `status_out` is non-null the raw word is also stored
+ * there (host pointer).  Returns FA_ERR_CUDA if the synchronisation itself failed. */
+int fa_read_device_status(int* status_out, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* fa_status_string(int status);
+
+/* Library ABI version (major*100 + minor). */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

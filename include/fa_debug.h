@@ -1,0 +1,36 @@
+/*
+ * fa_debug.h -- self-test entry points of libfa.so.  They exercise single hardware
+ * primitives the attention kernels are built from, so that a fault in a descriptor
+ * encoding or in the failure-detection path can be isolated on one tile.  They are not
+ * part of the attention method and have no counterpart on the source pages.
+ * Same conventions as fa.h: device pointers, asynchronous on `stream`, fa_status return,
+ * nothing launched on a non-zero return.
+ */
+#ifndef FA_DEBUG_H_
+#define FA_DEBUG_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* One CTA computes C = A * B with tcgen05.mma (bf16 in, fp32 accumulate in TMEM) and
+ * reads the accumulator back with tcgen05.ld.  A is [128][k] bf16 row-major; C is
+ * [128][n] fp32 row-major; n, k in {64, 128}.
+ *   mode 0: B is [n][k] bf16 row-major (K-major; C = A B^T), A and B in shared memory.
+ *   mode 1: B is [k][n] bf16 row-major (MN-major), A staged in TENSOR memory as packed
+ *           bf16 pairs (the P operand layout of the forward kernel).
+ *   mode 2: B is [k][n] bf16 row-major (MN-major), A in shared memory. */
+int fa_debug_umma_tile(const void* a, const void* b, float* c, int n, int k, int mode,
+                       void* stream);
+
+/* Launches one CTA whose only work is a bounded wait on an mbarrier that nothing ever
+ * arrives at.  The wait gives up after `timeout_ns` nanoseconds (1e3 .. 1e10), records
+ * FA_ERR_TIMEOUT in the device status word and the CTA exits normally.  Read the result
+ * with fa_read_device_status(). */
+int fa_debug_wait_timeout(long long timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_DEBUG_H_ */
