@@ -153,7 +153,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (check_shape(B, H, N, d, 1.0f) != FA_OK || d < 1) return 0;
   const size_t rows = static_cast<size_t>(B) * H * N;
-  return round_up(rows * d * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
+  const size_t padded = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128 * 128);
+  return round_up(rows * d * sizeof(float), 256) + 2 * round_up(padded * sizeof(float), 256);
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -183,9 +184,12 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   a.dq = dq;
   a.dk = dk;
   a.dv = dv;
-  a.dq_acc = static_cast<float*>(workspace);
-  a.delta = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                     round_up(rows * d * sizeof(float), 256));
+  const size_t padded = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128 * 128);
+  char* ws = static_cast<char*>(workspace);
+  a.dq_acc = reinterpret_cast<float*>(ws);
+  a.delta = reinterpret_cast<float*>(ws + round_up(rows * d * sizeof(float), 256));
+  a.lse2 = reinterpret_cast<float*>(ws + round_up(rows * d * sizeof(float), 256) +
+                                    round_up(padded * sizeof(float), 256));
   a.B = B;
   a.H = H;
   a.N = N;

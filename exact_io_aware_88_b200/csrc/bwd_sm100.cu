@@ -1,10 +1,519 @@
-// bwd_sm100.cu -- attention backward on sm_100a (placeholder until the kernels land).
+// bwd_sm100.cu -- attention backward on sm_100a.
+//
+// The backward pass does not read a stored P: it rebuilds S and P tile by tile from the
+// saved logsumexp, trading recomputation for memory traffic ("Flash Attention 2で打破する
+// ローカルLLMの「メモリの壁」", section タイリング（Tiling）と再計算（Recomputation）の仕組み).
+// Work is split along the key sequence (the second trick of "FlashAttention-2を読む",
+// section GPUの稼働率を高める三つの工夫): one CTA owns a 128-row K/V tile and walks the
+// query tiles that can see it.
+//
+// Three kernels, all on the caller's stream:
+//  1. bwd_pre    D = rowsum(dO o O) (fp32) and lse2 = LSE*log2(e), both stored padded to a
+//                multiple of 128 rows; clears the fp32 dQ accumulator.          (HBM-bound)
+//  2. bwd_main   per (b, h, kv tile j), for each visible query tile i:
+//                  S^T  = K_j Q_i^T          (tcgen05, TMEM)
+//                  dP^T = V_j dO_i^T         (tcgen05, TMEM)
+//                  P^T  = exp2(S^T*scale*log2e - lse2_i)       (compute warps; bf16 -> TMEM)
+//                  dS^T = P^T o (dP^T - D_i)                  (compute warps; bf16 -> smem)
+//                  dV_j += P^T dO_i,  dK_j += dS^T Q_i          (tcgen05, TMEM accumulators)
+//                  dQ_i  = dS K_j  -> fp32 vector atomics into the accumulator (dQ warps)
+//                epilogue: dK_j*scale, dV_j -> bf16.
+//  3. dq_convert dq = bf16(scale * dQacc).                                     (HBM-bound)
+//
+// bwd_main CTA = 10 warps: 0-3 compute (thread t owns key row t = TMEM lane t), 4 TMA
+// producer, 5 TMEM allocator + MMA issuer, 6-9 dQ drain (thread owns query row = TMEM lane).
+// TMEM (512 columns): dK [0,D), dV [D,2D), S^T/P^T [2D,2D+128), dP^T and then dQ
+// [2D+128,2D+256).
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
 
 #include "launch.h"
+#include "ptx.cuh"
 
 namespace fa {
+namespace bwd {
 
-cudaError_t launch_bwd_sm100(const BwdArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+constexpr int BM = 128;  // key rows per CTA tile (MMA M)
+constexpr int BN = 128;  // query rows per step
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct Cfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kChunkBytes = 128 * 128;  // one TMA box: 128 rows x 128 B
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kQStages = 2;
+  static constexpr int kDOStages = (D == 128) ? 1 : 2;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kTileBytes;
+  static constexpr int kOffQ = kOffV + kTileBytes;
+  static constexpr int kOffDO = kOffQ + kQStages * kTileBytes;
+  static constexpr int kOffDS = kOffDO + kDOStages * kTileBytes;  // dS^T: 2 chunks x 16 KB
+  static constexpr int kOffVec = kOffDS + 2 * kChunkBytes;         // lse2 / D per q stage
+  static constexpr int kVecBytes = kQStages * 2 * BN * 4;
+  static constexpr int kOffBar = kOffVec + kVecBytes;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+  static constexpr uint32_t kColDK = 0;
+  static constexpr uint32_t kColDV = D;
+  static constexpr uint32_t kColS = 2 * D;
+  static constexpr uint32_t kColDP = 2 * D + 128;
+};
+
+struct Bars {
+  uint64_t kv_full;
+  uint64_t q_full[2], q_empty[2];
+  uint64_t do_full[2], do_empty[2];
+  uint64_t s_full, dp_full, ds_ready, dq_full, dq_empty, dkdv_done, drain;
+  uint32_t tmem_base;
+  Abort abort;
+};
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const float* __restrict__ lse2, const float* __restrict__ delta,
+                    float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk,
+                    __nv_bfloat16* __restrict__ dv, int B, int H, int N, int n_pad,
+                    float scale, float scale_log2, int num_kvtiles, int* status,
+                    uint64_t timeout_ns) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Work unit (b, h, kv tile j); heads major for L2 reuse of Q/dO; under the causal mask
+  // low j (the most query tiles) first.
+  const int bh = blockIdx.x / num_kvtiles;
+  const int j = blockIdx.x % num_kvtiles;
+  const int b = bh / H, h = bh % H;
+  const int k0 = j * BM;
+  const int nq_total = (N + BN - 1) / BN;
+  const int i_begin = CAUSAL ? j : 0;
+  const int nq = nq_total - i_begin;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->q_full[s], 1);
+      mbar_init(&bars->q_empty[s], 1);
+      mbar_init(&bars->do_full[s], 1);
+      mbar_init(&bars->do_empty[s], 1);
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->dp_full, 1);
+    mbar_init(&bars->ds_ready, 128);
+    mbar_init(&bars->dq_full, 1);
+    mbar_init(&bars->dq_empty, 128);
+    mbar_init(&bars->dkdv_done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort.flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = bars->tmem_base;
+  Abort* ab = &bars->abort;
+
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sDO = smem + C::kOffDO;
+  uint8_t* sDS = smem + C::kOffDS;
+  float* sVec = reinterpret_cast<float*>(smem + C::kOffVec);  // [stage][lse2 | D][128]
+  const size_t vec_base = static_cast<size_t>(bh) * n_pad;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_do);
+      const uint64_t pol_kv = policy_evict_first();
+      const uint64_t pol_q = policy_evict_last();
+      mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTileBytes);
+      for (int c = 0; c < C::kChunks; ++c) {
+        tma_load_4d(sK + c * C::kChunkBytes, &tm_k, &bars->kv_full, c * 64, h, k0, b, pol_kv);
+        tma_load_4d(sV + c * C::kChunkBytes, &tm_v, &bars->kv_full, c * 64, h, k0, b, pol_kv);
+      }
+      int issued_q = 0, issued_do = 0;
+      for (int n = 0; n < nq; ++n) {
+        const int i = i_begin + n;
+        const int sq = n % C::kQStages;
+        if (n >= C::kQStages &&
+            !mbar_wait(&bars->q_empty[sq], ((n / C::kQStages) - 1) & 1, ab, status, timeout_ns))
+          break;
+        mbar_arrive_expect_tx(&bars->q_full[sq], C::kTileBytes + 2 * BN * 4);
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_4d(sQ + sq * C::kTileBytes + c * C::kChunkBytes, &tm_q, &bars->q_full[sq],
+                      c * 64, h, i * BN, b, pol_q);
+        bulk_load(sVec + sq * 2 * BN, lse2 + vec_base + i * BN, BN * 4, &bars->q_full[sq]);
+        bulk_load(sVec + sq * 2 * BN + BN, delta + vec_base + i * BN, BN * 4, &bars->q_full[sq]);
+        issued_q = n + 1;
+        const int sd = n % C::kDOStages;
+        if (n >= C::kDOStages &&
+            !mbar_wait(&bars->do_empty[sd], ((n / C::kDOStages) - 1) & 1, ab, status, timeout_ns))
+          break;
+        mbar_arrive_expect_tx(&bars->do_full[sd], C::kTileBytes);
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_4d(sDO + sd * C::kTileBytes + c * C::kChunkBytes, &tm_do, &bars->do_full[sd],
+                      c * 64, h, i * BN, b, pol_q);
+        issued_do = n + 1;
+      }
+      // Drain every copy into shared memory before the CTA may exit.
+      Abort local{0};
+      mbar_wait(&bars->kv_full, 0, &local, status, timeout_ns);
+      for (int n = max(0, issued_q - C::kQStages); n < issued_q; ++n)
+        mbar_wait(&bars->q_full[n % C::kQStages], (n / C::kQStages) & 1, &local, status, timeout_ns);
+      for (int n = max(0, issued_do - C::kDOStages); n < issued_do; ++n)
+        mbar_wait(&bars->do_full[n % C::kDOStages], (n / C::kDOStages) & 1, &local, status,
+                  timeout_ns);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_sdp = idesc_bf16_f32(BM, BN, 0, 0);  // K_j Q_i^T, V_j dO_i^T
+      constexpr uint32_t id_dkdv = idesc_bf16_f32(BM, D, 0, 1);  // P^T dO_i, dS^T Q_i
+      constexpr uint32_t id_dq = idesc_bf16_f32(BN, D, 1, 1);    // dS K_j (A MN-major)
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ),
+                     aDO = smem_u32(sDO), aDS = smem_u32(sDS);
+      bool ok = mbar_wait(&bars->kv_full, 0, ab, status, timeout_ns);
+      for (int n = 0; ok && n < nq; ++n) {
+        const int sq = n % C::kQStages, sd = n % C::kDOStages;
+        if (!mbar_wait(&bars->q_full[sq], (n / C::kQStages) & 1, ab, status, timeout_ns)) break;
+        tc_fence_after();
+        const uint32_t qb = aQ + sq * C::kTileBytes, dob = aDO + sd * C::kTileBytes;
+        // S^T = K_j Q_i^T  (both K-major over the head dim)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+          umma_ss(tbase + C::kColS, sdesc_sw128(aK + off, 16, 1024), sdesc_sw128(qb + off, 16, 1024),
+                  id_sdp, kk > 0);
+        }
+        umma_commit(&bars->s_full);
+        if (!mbar_wait(&bars->do_full[sd], (n / C::kDOStages) & 1, ab, status, timeout_ns)) break;
+        if (n > 0 && !mbar_wait(&bars->dq_empty, (n - 1) & 1, ab, status, timeout_ns)) break;
+        tc_fence_after();
+        // dP^T = V_j dO_i^T  (columns previously holding dQ_{i-1}, now drained)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+          umma_ss(tbase + C::kColDP, sdesc_sw128(aV + off, 16, 1024),
+                  sdesc_sw128(dob + off, 16, 1024), id_sdp, kk > 0);
+        }
+        umma_commit(&bars->dp_full);
+        if (!mbar_wait(&bars->ds_ready, n & 1, ab, status, timeout_ns)) break;
+        tc_fence_after();
+        // dV_j += P^T dO_i   (A = P^T from TMEM, B = dO_i MN-major over the query index)
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_ts(tbase + C::kColDV, tbase + C::kColS + kk * 8,
+                  sdesc_sw128(dob + kk * 2048, C::kChunkBytes, 1024), id_dkdv, (n > 0 || kk > 0));
+        umma_commit(&bars->do_empty[sd]);
+        // dK_j += dS^T Q_i   (A = dS^T K-major over the query index, B = Q_i MN-major)
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+          umma_ss(tbase + C::kColDK, sdesc_sw128(aDS + aoff, 16, 1024),
+                  sdesc_sw128(qb + kk * 2048, C::kChunkBytes, 1024), id_dkdv, (n > 0 || kk > 0));
+        }
+        // dQ_i = dS K_j   (A = dS: the same smem tile read MN-major; B = K_j MN-major)
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          umma_ss(tbase + C::kColDP, sdesc_sw128(aDS + kk * 2048, C::kChunkBytes, 1024),
+                  sdesc_sw128(aK + kk * 2048, C::kChunkBytes, 1024), id_dq, kk > 0);
+        umma_commit(&bars->dq_full);
+        umma_commit(&bars->q_empty[sq]);
+      }
+      umma_commit(&bars->dkdv_done);
+      umma_commit(&bars->drain);
+      Abort local{0};
+      mbar_wait(&bars->drain, 0, &local, status, timeout_ns);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------------ compute warps
+    const int t = threadIdx.x;  // key row within the tile == TMEM lane
+    const int key = k0 + t;
+    const uint32_t lane_base = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+    bool ok = true;
+    for (int n = 0; n < nq; ++n) {
+      const int i = i_begin + n;
+      const int q0 = i * BN;
+      const int sq = n % C::kQStages;
+      const float* sL = sVec + sq * 2 * BN;
+      const float* sD = sL + BN;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, n & 1, ab, status, timeout_ns));
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->q_full[sq], (n / C::kQStages) & 1, ab, status,
+                                             timeout_ns));
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, n & 1, ab, status, timeout_ns));
+      if (!ok) break;
+      tc_fence_after();
+      // Columns c with q0 + c < key are masked (query before key) on diagonal tiles; keys
+      // and queries past N are masked on tail tiles.
+      const bool row_dead = key >= N;
+      const int first_vis = CAUSAL ? key - q0 : 0;  // first visible column
+      const int last_vis = N - 1 - q0;               // last existing column
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {  // 32 query columns at a time
+        uint32_t su[32], du[32];
+        tmem_ld32(lane_base + C::kColS + qq * 32, su);
+        tmem_ld32(lane_base + C::kColDP + qq * 32, du);
+        uint32_t ppk[16], dpk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const int c = qq * 32 + e;
+          const float4 l4 = *reinterpret_cast<const float4*>(sL + c);
+          const float4 d4 = *reinterpret_cast<const float4*>(sD + c);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+          const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+          float p[4], ds[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            p[u] = ex2_approx(fmaf(__uint_as_float(su[e + u]), scale_log2, -lv[u]));
+            if (row_dead || c + u < first_vis || c + u > last_vis) p[u] = 0.f;
+            ds[u] = p[u] * (__uint_as_float(du[e + u]) - dv4[u]);
+          }
+          ppk[e / 2] = pack_bf16x2(p[0], p[1]);
+          ppk[e / 2 + 1] = pack_bf16x2(p[2], p[3]);
+          dpk[e / 2] = pack_bf16x2(ds[0], ds[1]);
+          dpk[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+        }
+        // P^T (bf16 pairs) into columns [16qq, 16qq+16) of the S^T region, whose S^T values
+        // were consumed by this or an earlier quarter.
+        tmem_st16(lane_base + C::kColS + qq * 16, ppk);
+        // dS^T row t, query columns [32qq, 32qq+32): chunk qq/2, 16-byte pieces 4(qq%2)..+3.
+        uint8_t* chunk = sDS + (qq >> 1) * C::kChunkBytes;
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc)
+          *reinterpret_cast<uint4*>(chunk + sw128_offset(t, (qq & 1) * 4 + pc)) =
+              make_uint4(dpk[4 * pc], dpk[4 * pc + 1], dpk[4 * pc + 2], dpk[4 * pc + 3]);
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars->ds_ready);
+    }
+    // ---------------------------------------------------------------- dK / dV epilogue
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->dkdv_done, 0, ab, status, timeout_ns));
+    if (ok) {
+      tc_fence_after();
+      const size_t orow = ((static_cast<size_t>(b) * N + key) * H + h) * D;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which == 0 ? C::kColDK : C::kColDV;
+        const float mul = which == 0 ? scale : 1.f;
+        __nv_bfloat16* dst = (which == 0 ? dk : dv) + orow;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t u[32];
+          tmem_ld32(lane_base + col + c * 32, u);
+          if (key < N) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              d4[v4] = make_uint4(
+                  pack_bf16x2(__uint_as_float(u[8 * v4 + 0]) * mul, __uint_as_float(u[8 * v4 + 1]) * mul),
+                  pack_bf16x2(__uint_as_float(u[8 * v4 + 2]) * mul, __uint_as_float(u[8 * v4 + 3]) * mul),
+                  pack_bf16x2(__uint_as_float(u[8 * v4 + 4]) * mul, __uint_as_float(u[8 * v4 + 5]) * mul),
+                  pack_bf16x2(__uint_as_float(u[8 * v4 + 6]) * mul, __uint_as_float(u[8 * v4 + 7]) * mul));
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ dQ drain warps
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = quarter * 32 + lane;  // query row within the tile
+    const uint32_t lane_base = tbase + (static_cast<uint32_t>(quarter * 32) << 16);
+    for (int n = 0; n < nq; ++n) {
+      const int q = (i_begin + n) * BN + r;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_full, n & 1, ab, status, timeout_ns));
+      if (!ok) break;
+      tc_fence_after();
+      float* dst = dq_acc + (static_cast<size_t>(bh) * N + q) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld32(lane_base + C::kColDP + c * 32, u);
+        if (q < N) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            atomicAdd(reinterpret_cast<float4*>(dst + c * 32 + 4 * v),
+                      make_float4(__uint_as_float(u[4 * v]), __uint_as_float(u[4 * v + 1]),
+                                  __uint_as_float(u[4 * v + 2]), __uint_as_float(u[4 * v + 3])));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->dq_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) {
+    __syncwarp();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+// D[bh][n] = sum_c dO[b,n,h,c] * O[b,n,h,c];  lse2[bh][n] = lse[bh][n] * log2(e);  zero rows
+// n in [N, n_pad); dQacc = 0.  Threads per row: D/8 (one 16-byte vector each).
+template <int D>
+__global__ void __launch_bounds__(256)
+    bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+                   const float* __restrict__ lse, float* __restrict__ delta,
+                   float* __restrict__ lse2, float* __restrict__ dq_acc, int B, int H, int N,
+                   int n_pad, long long acc_vec4, int row_blocks) {
+  constexpr int kTPR = D / 8;           // threads per row
+  constexpr int kRowsPerBlock = 256 / kTPR;
+  if (static_cast<int>(blockIdx.x) < row_blocks) {
+    const long long rows = static_cast<long long>(B) * N * H;  // rows in memory order (b, n, h)
+    const long long row = static_cast<long long>(blockIdx.x) * kRowsPerBlock + threadIdx.x / kTPR;
+    const int part = threadIdx.x % kTPR;
+    float acc = 0.f;
+    if (row < rows) {
+      const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
+      const uint4 g = *reinterpret_cast<const uint4*>(dO + row * D + part * 8);
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fa = __bfloat1622float2(a2[e]);
+        const float2 fg = __bfloat1622float2(g2[e]);
+        acc = fmaf(fa.x, fg.x, acc);
+        acc = fmaf(fa.y, fg.y, acc);
+      }
+    }
+#pragma unroll
+    for (int off = kTPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (row < rows && part == 0) {
+      const int h = static_cast<int>(row % H);
+      const long long bn = row / H;
+      const int n = static_cast<int>(bn % N);
+      const int b = static_cast<int>(bn / N);
+      const size_t bhn = (static_cast<size_t>(b) * H + h);
+      delta[bhn * n_pad + n] = acc;
+      lse2[bhn * n_pad + n] = lse[bhn * N + n] * kLog2e;
+    }
+    // Padding rows [N, n_pad) of every (b, h): written by the first blocks.
+    const long long pad_rows = static_cast<long long>(B) * H * (n_pad - N);
+    for (long long p = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; p < pad_rows;
+         p += static_cast<long long>(row_blocks) * 256) {
+      const long long bhi = p / (n_pad - N);
+      const int n = N + static_cast<int>(p % (n_pad - N));
+      delta[bhi * n_pad + n] = 0.f;
+      lse2[bhi * n_pad + n] = 0.f;
+    }
+  } else {
+    // Zero the dQ accumulator.
+    const long long nblk = static_cast<long long>(gridDim.x) - row_blocks;
+    float4* acc4 = reinterpret_cast<float4*>(dq_acc);
+    for (long long p = (static_cast<long long>(blockIdx.x) - row_blocks) * 256 + threadIdx.x;
+         p < acc_vec4; p += nblk * 256)
+      acc4[p] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// dq[b][n][h][:] = bf16(scale * dQacc[b][h][n][:]).  One thread per 8 output elements.
+template <int D>
+__global__ void __launch_bounds__(256)
+    dq_convert_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dq, int B,
+                      int H, int N, float scale) {
+  constexpr int kTPR = D / 8;
+  const long long rows = static_cast<long long>(B) * N * H;
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long row = gid / kTPR;
+  const int part = static_cast<int>(gid % kTPR);
+  if (row >= rows) return;
+  const int h = static_cast<int>(row % H);
+  const long long bn = row / H;
+  const int n = static_cast<int>(bn % N);
+  const long long b = bn / N;
+  const float4* src = reinterpret_cast<const float4*>(
+      dq_acc + ((static_cast<size_t>(b) * H + h) * N + n) * D + part * 8);
+  const float4 x = src[0], y = src[1];
+  *reinterpret_cast<uint4*>(dq + row * D + part * 8) =
+      make_uint4(pack_bf16x2(x.x * scale, x.y * scale), pack_bf16x2(x.z * scale, x.w * scale),
+                 pack_bf16x2(y.x * scale, y.y * scale), pack_bf16x2(y.z * scale, y.w * scale));
+}
+
+template <int D, bool CAUSAL>
+static cudaError_t launch_t(const BwdArgs& a, cudaStream_t st) {
+  using C = Cfg<D>;
+  const int n_pad = (a.N + 127) / 128 * 128;
+  const size_t rows = static_cast<size_t>(a.B) * a.H * a.N;
+  float* lse2 = a.lse2;
+
+  // 1. preprocess
+  {
+    constexpr int kRowsPerBlock = 256 / (D / 8);
+    const long long row_blocks = (static_cast<long long>(rows) + kRowsPerBlock - 1) / kRowsPerBlock;
+    const long long acc_vec4 = static_cast<long long>(rows) * D / 4;
+    const long long zero_blocks = std::min<long long>((acc_vec4 + 255) / 256, 4LL * a.num_sms * 8);
+    const long long grid = row_blocks + zero_blocks;
+    if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    bwd_pre_kernel<D><<<static_cast<unsigned>(grid), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse,
+        a.delta, lse2, a.dq_acc, a.B, a.H, a.N, n_pad, acc_vec4, static_cast<int>(row_blocks));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  // 2. main
+  {
+    auto kern = bwd_main_kernel<D, CAUSAL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int num_kvtiles = (a.N + BM - 1) / BM;
+    const long long grid = static_cast<long long>(a.B) * a.H * num_kvtiles;
+    kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, st>>>(
+        a.tm_q, a.tm_k, a.tm_v, a.tm_do, lse2, a.delta, a.dq_acc,
+        static_cast<__nv_bfloat16*>(a.dk), static_cast<__nv_bfloat16*>(a.dv), a.B, a.H, a.N, n_pad,
+        a.scale, a.scale * kLog2e, num_kvtiles, a.status, kDefaultWaitTimeoutNs);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  // 3. dQ conversion
+  {
+    const long long threads = static_cast<long long>(rows) * (D / 8);
+    const long long grid = (threads + 255) / 256;
+    dq_convert_kernel<D><<<static_cast<unsigned>(grid), 256, 0, st>>>(
+        a.dq_acc, static_cast<__nv_bfloat16*>(a.dq), a.B, a.H, a.N, a.scale);
+    return cudaGetLastError();
+  }
+}
+
+}  // namespace bwd
+
+cudaError_t launch_bwd_sm100(const BwdArgs& a, cudaStream_t s) {
+  if (a.d == 64) return a.causal ? bwd::launch_t<64, true>(a, s) : bwd::launch_t<64, false>(a, s);
+  return a.causal ? bwd::launch_t<128, true>(a, s) : bwd::launch_t<128, false>(a, s);
+}
 
 }  // namespace fa

@@ -29,7 +29,8 @@ struct BwdArgs {
   const float* lse;
   void *dq, *dk, *dv;
   float* dq_acc;  // [B][H][N][d] fp32 workspace
-  float* delta;   // [B][H][N] fp32 workspace
+  float* delta;   // [B][H][n_pad] fp32 workspace, n_pad = N rounded up to 128
+  float* lse2;    // [B][H][n_pad] fp32 workspace: lse * log2(e)
   int B, H, N, d, causal;
   float scale;
   int* status;

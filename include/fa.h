@@ -59,16 +59,17 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            int B, int H, int N, int d, int causal, float scale, void* stream);
 
 /* Bytes of device workspace fa_bwd needs for this problem: an fp32 dQ accumulator
- * (B*H*N*d floats) and the fp32 row statistic D (B*H*N floats), each 256-byte aligned.
- * Returns 0 if the arguments are invalid. */
+ * (B*H*N*d floats), then the fp32 row statistic D and the base-2 logsumexp, each
+ * B*H*Np floats with Np = N rounded up to a multiple of 128; every part starts on a
+ * 256-byte boundary.  Returns 0 if the arguments are invalid. */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
 /* Backward pass.  Inputs are the forward's q, k, v, its outputs o and lse, and the
  * upstream gradient dO (all [B][N][H][d] bf16 except lse, which must be 16-byte
  * aligned here).  Writes dq, dk, dv
  * ([B][N][H][d] bf16).  `workspace` is caller-owned device memory of at least
- * fa_bwd_workspace_bytes(B, H, N, d) bytes; its contents on entry are ignored and on
- * return are unspecified.  d must be 64 or 128.
+ * fa_bwd_workspace_bytes(B, H, N, d) bytes, 256-byte aligned; its contents on entry are
+ * ignored and on return are unspecified.  d must be 64 or 128.
  * Steps: D = rowsum(dO o O) with dQ-accumulator clearing; per key/value tile, recompute
  * S^T and P^T from lse, dP^T = V dO^T, dS^T = P^T o (dP^T - D); dV += P^T dO and
  * dK += dS^T Q accumulate in TMEM; dQ += dS K is reduced in fp32 into the workspace

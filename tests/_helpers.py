@@ -24,3 +24,12 @@ def to_np(t: torch.Tensor):
 
 def cuda(tensors, names):
     return [tensors[n].to("cuda:0") for n in names]
+
+
+def grad_err(x, ref):
+    """Relative L2 error; where the exact gradient is identically zero (e.g. dQ and dK of a
+    single-key problem, whose softmax is constant) the max-abs error is returned instead."""
+    n = float(np.linalg.norm(ref))
+    if n == 0.0:
+        return float(np.abs(np.asarray(x)).max())
+    return rel_l2(x, ref)

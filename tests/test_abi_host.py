@@ -47,7 +47,8 @@ def test_workspace_size_formula(fa):
         return (x + 255) // 256 * 256
     for B, H, N, d in [(1, 16, 4096, 128), (2, 3, 1000, 64), (1, 1, 1, 64)]:
         rows = B * H * N
-        assert fa.fa_bwd_workspace_bytes(B, H, N, d) == up(rows * d * 4) + up(rows * 4)
+        padded = B * H * ((N + 127) // 128 * 128)
+        assert fa.fa_bwd_workspace_bytes(B, H, N, d) == up(rows * d * 4) + 2 * up(padded * 4)
     assert fa.fa_bwd_workspace_bytes(0, 1, 1, 64) == 0
     assert fa.fa_bwd_workspace_bytes(1, 1, -5, 64) == 0
 
