@@ -1,0 +1,419 @@
+"""Throughput benchmark of the attention hot path (forward + backward) on B200.
+
+One step = one pass of the whole hot path over one batch of the workload
+"fwdbwd_d128": B*N = 16384 tokens, H = 16 heads of dim 128, causal, bf16, with the
+sequence length N = 16384 (B = 1) by default:
+    fa_fwd -> fa_bwd_preprocess -> fa_bwd_kv -> fa_bwd_dq_convert
+Throughput is attention TFLOPS: 4*B*H*N^2*d (halved under the causal mask) for the
+forward plus 2.5x that for the backward, over the device time of the timed steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--N 16384]
+
+Under torchrun (N > 1) every rank runs its own copy of the workload (independent
+problems, no collective on the data path: weak scaling); the step time is the max over
+ranks.  Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle on
+a bounded sample instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+METRIC = "attention fwd/bwd TFLOPS on 1 B200 vs BF16 tensor-core peak (fraction of roofline)"
+UNIT = "TFLOPS"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 4  # fwd, bwd_pre, bwd_main, dq_convert
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_env():
+    """(rank, world_size, local_rank) from the torchrun environment (1 process if unset)."""
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def init_dist(world: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar (the step time) over all ranks; identity on one rank."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ measurement helpers
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": ["no samples"]}
+        loaded = [x for x in sm if x > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_id(dev) -> str:
+    """nvidia-smi selector of the device torch calls `dev` (its UUID; robust to
+    CUDA_VISIBLE_DEVICES renumbering)."""
+    import torch
+    props = torch.cuda.get_device_properties(dev)
+    u = str(getattr(props, "uuid", ""))
+    if u:
+        return u if u.startswith("GPU-") else "GPU-" + u
+    return str(dev.index or 0)
+
+
+def kernel_source_hash() -> str:
+    p = os.path.join(ROOT, "exact_io_aware_88_b200", "csrc", "bwd_sm100.cu")
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary of `kernel` on `workload`,
+    or None when there is none or the kernel source changed since it was captured."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", txt)
+    if not m or not h or h.group(1) != kernel_source_hash():
+        return None
+    return float(m.group(1))
+
+
+# ------------------------------------------------------------------ the CUDA path
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = init_dist(world, "nccl")
+    from exact_io_aware_88_b200 import fa
+
+    w = workload(args.N)
+    t = synthetic.draw_workload(w, with_grad=True)
+    B, N, H, d = w.B, w.N, w.H, w.d
+    q, k, v, dO = (t[n].to(dev) for n in ("q", "k", "v", "dO"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa.fa_bwd_workspace_bytes(B, H, N, d)
+    ws = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+    sc = w.scale
+
+    def check(rc, fn):
+        if rc != 0:
+            raise RuntimeError(f"{fn} failed: {fa.status_string(rc)}")
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        check(fa.fa_fwd(q, k, v, o, lse, B, H, N, d, w.causal, sc, stream), "fa_fwd")
+        if ev is not None:
+            ev[1].record(stream)
+        check(fa.fa_bwd_preprocess(o, lse, dO, B, H, N, d, ws, ws_bytes, stream), "fa_bwd_preprocess")
+        if ev is not None:
+            ev[2].record(stream)
+        check(fa.fa_bwd_kv(q, k, v, dO, dk, dv, B, H, N, d, w.causal, sc, ws, ws_bytes, stream),
+              "fa_bwd_kv")
+        if ev is not None:
+            ev[3].record(stream)
+        check(fa.fa_bwd_dq_convert(dq, B, H, N, d, sc, ws, ws_bytes, stream), "fa_bwd_dq_convert")
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    check(fa.fa_read_device_status(stream), "device status")
+
+    # ---- device-resident timed region: K steps, events around each kernel.
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(gpu_id(dev)) as clk:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    total_ms = max_over_ranks(start.elapsed_time(end), world, dev)
+    clocks = clk.summary()
+    check(fa.fa_read_device_status(stream), "device status")
+    per_kernel = {nm: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+                  for i, nm in enumerate(["fwd", "bwd_pre", "bwd_main", "dq_convert"])}
+
+    # ---- end to end through the public API with host buffers (pinned), copies included.
+    hq, hk, hv, hdO = (t[n].pin_memory() for n in ("q", "k", "v", "dO"))
+    ho, hdq, hdk, hdv = (torch.empty_like(x).pin_memory() for x in (hq, hq, hk, hv))
+    hlse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        for dst, src in ((q, hq), (k, hk), (v, hv), (dO, hdO)):
+            dst.copy_(src, non_blocking=True)
+        check(fa.fa_fwd(q, k, v, o, lse, B, H, N, d, w.causal, sc, stream), "fa_fwd")
+        check(fa.fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, w.causal, sc, ws, ws_bytes,
+                        stream), "fa_bwd")
+        for dst, src in ((ho, o), (hlse, lse), (hdq, dq), (hdk, dk), (hdv, dv)):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdO))
+    d2h = sum(x.numel() * x.element_size() for x in (ho, hlse, hdq, hdk, hdv))
+
+    ms_step = total_ms / args.steps
+    flops = w.fwd_flops() + w.bwd_flops()
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    peaks, peak_src = measured_peaks()
+    peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    main_tflops = w.bwd_flops() / (per_kernel["bwd_main"] * 1e-3) / 1e12
+    fwd_tflops = w.fwd_flops() / (per_kernel["fwd"] * 1e-3) / 1e12
+    wl = f"fwdbwd_d128_N{N}"
+    traffic = profiled_traffic("bwd_main", wl)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, t)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"{w.name}: B={B} N={N} H={H} d={d} causal bf16, "
+                                   "q/k/v/dO ~ N(0,1) seed 1003",
+                       "B": B, "N": N, "H": H, "d": d, "causal": True,
+                       "tokens_per_gpu": B * N,
+                       "parallelism": f"replicas x{world} (independent problems per GPU)",
+                       "l2": "no flush: inputs (q,k,v,o,dO = %d MiB) exceed the 126 MB L2"
+                             % (5 * q.numel() * 2 // 2 ** 20)},
+            "breakdown": {
+                "fwd_ms": round(per_kernel["fwd"], 4), "bwd_pre_ms": round(per_kernel["bwd_pre"], 4),
+                "bwd_main_ms": round(per_kernel["bwd_main"], 4),
+                "dq_convert_ms": round(per_kernel["dq_convert"], 4),
+                "fwd_tflops": round(fwd_tflops, 1), "bwd_main_tflops": round(main_tflops, 1),
+                "fwd_frac_of_burst_peak": round(fwd_tflops / peak_burst, 4),
+                "bwd_frac_of_burst_peak": round(w.bwd_flops() / ((per_kernel["bwd_pre"] + per_kernel["bwd_main"] + per_kernel["dq_convert"]) * 1e-3) / 1e12 / peak_burst, 4),
+            },
+            "roofline": {"kernel": "bwd_main (fa_bwd_kv)", "bound": "tensor",
+                         "achieved": round(main_tflops, 1), "peak": peak_sus, "unit": "TFLOP/s",
+                         "frac": round(main_tflops / peak_sus, 4),
+                         "peak_kind": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                         "frac_of_burst_peak": round(main_tflops / peak_burst, 4),
+                         "traffic": traffic},
+            "clocks": clocks,
+            "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms, 3)},
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def workload(N: int):
+    if N == 65536:
+        return synthetic.long_context()
+    return synthetic.fwdbwd(N)
+
+
+# ------------------------------------------------------------------ the oracle on the host
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(t, w, b: int, h: int, n_rows: int):
+    """fwd + bwd of one head of the workload, truncated to its first n_rows positions.
+    Under the causal mask that prefix is itself an exact attention problem.  Returns
+    (seconds, algorithmic FLOPs of the sample)."""
+    import oracle
+    Q, K, V, dO = (synthetic.to_f64(t[n][b, :n_rows, h]) for n in ("q", "k", "v", "dO"))
+    t0 = time.perf_counter()
+    oracle.forward_head(Q, K, V, w.scale, True)
+    oracle.backward_head(Q, K, V, dO, w.scale, True)
+    dt = time.perf_counter() - t0
+    flops = 3.5 * 4.0 * n_rows * n_rows * w.d / 2
+    return dt, flops
+
+
+def cpu_baseline(w, t):
+    n_rows = min(w.N, 16384)
+    dt, flops = oracle_sample(t, w, 0, 0, n_rows)
+    return {"value": round(flops / dt / 1e12, 5), "unit": UNIT, "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"head (b=0,h=0) of the workload, first {n_rows} positions, fwd+bwd "
+                      f"(fp64 numpy, S and P materialised); {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = workload(args.N)
+    t = synthetic.draw(w.B, w.N, w.H, w.d, w.seed, "bf16", with_grad=True)
+    n_rows = 4096
+    for s in range(args.warmup):
+        oracle_sample(t, w, 0, s % w.H, n_rows)
+    secs, fl = 0.0, 0.0
+    for s in range(args.steps):
+        dt, f = oracle_sample(t, w, 0, s % w.H, n_rows)
+        secs += dt
+        fl += f
+    value = fl / secs / 1e12
+    cores = blas_threads()
+    sample = (f"per step: one head of the workload truncated to its first {n_rows} positions "
+              "(an exact causal sub-problem), fwd+bwd, fp64 numpy oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * secs / args.steps, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{w.name}: B={w.B} N={w.N} H={w.H} d={w.d} causal bf16 inputs",
+                       "B": w.B, "N": w.N, "H": w.H, "d": w.d, "causal": True},
+            "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--N", type=int, default=16384, choices=[1024, 2048, 4096, 8192, 16384, 65536])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local_rank = dist_env()
+    if world != args.gpus and world > 1:
+        print(f"warning: WORLD_SIZE={world} but --gpus={args.gpus}", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

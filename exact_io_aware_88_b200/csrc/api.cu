@@ -157,48 +157,107 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   return round_up(rows * d * sizeof(float), 256) + 2 * round_up(padded * sizeof(float), 256);
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-           const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal,
-           float scale, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+enum BwdStage { kStagePre = 1, kStageMain = 2, kStageConvert = 4 };
+
+// Validates the arguments the requested stages use and fills `a`.  Pointers a stage does
+// not use may be null.
+int bwd_prepare(int stages, const void* q, const void* k, const void* v, const void* o,
+                const float* lse, const void* dO, void* dq, void* dk, void* dv, int B, int H,
+                int N, int d, int causal, float scale, void* workspace, size_t workspace_bytes,
+                fa::BwdArgs* a) {
+  const bool pre = stages & kStagePre, mid = stages & kStageMain, cvt = stages & kStageConvert;
+  if ((pre && (!o || !lse || !dO)) || (mid && (!q || !k || !v || !dO || !dk || !dv)) ||
+      (cvt && !dq))
+    return FA_ERR_INVALID_ARG;
   int rc = check_shape(B, H, N, d, scale);
   if (rc) return rc;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
-      !aligned(dO, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
-      !aligned(lse, 16))
+  if ((pre && (!aligned(o, 16) || !aligned(dO, 16) || !aligned(lse, 16))) ||
+      (mid && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dO, 16) ||
+               !aligned(dk, 16) || !aligned(dv, 16))) ||
+      (cvt && !aligned(dq, 16)))
     return FA_ERR_MISALIGNED;
   const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
   if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return FA_ERR_MISALIGNED;
   DeviceInfo di;
   if ((rc = device_info(&di))) return rc;
-  fa::BwdArgs a;
-  if ((rc = encode_bnhd(&a.tm_q, q, B, N, H, d)) || (rc = encode_bnhd(&a.tm_k, k, B, N, H, d)) ||
-      (rc = encode_bnhd(&a.tm_v, v, B, N, H, d)) || (rc = encode_bnhd(&a.tm_do, dO, B, N, H, d)))
+  if (mid && ((rc = encode_bnhd(&a->tm_q, q, B, N, H, d)) ||
+              (rc = encode_bnhd(&a->tm_k, k, B, N, H, d)) ||
+              (rc = encode_bnhd(&a->tm_v, v, B, N, H, d)) ||
+              (rc = encode_bnhd(&a->tm_do, dO, B, N, H, d))))
     return rc;
   const size_t rows = static_cast<size_t>(B) * H * N;
-  a.o = o;
-  a.dO = dO;
-  a.lse = lse;
-  a.dq = dq;
-  a.dk = dk;
-  a.dv = dv;
   const size_t padded = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128 * 128);
   char* ws = static_cast<char*>(workspace);
-  a.dq_acc = reinterpret_cast<float*>(ws);
-  a.delta = reinterpret_cast<float*>(ws + round_up(rows * d * sizeof(float), 256));
-  a.lse2 = reinterpret_cast<float*>(ws + round_up(rows * d * sizeof(float), 256) +
-                                    round_up(padded * sizeof(float), 256));
-  a.B = B;
-  a.H = H;
-  a.N = N;
-  a.d = d;
-  a.causal = causal ? 1 : 0;
-  a.scale = scale;
-  a.status = di.status;
-  a.num_sms = di.num_sms;
-  return from_cuda(fa::launch_bwd_sm100(a, static_cast<cudaStream_t>(stream)));
+  a->o = o;
+  a->dO = dO;
+  a->lse = lse;
+  a->dq = dq;
+  a->dk = dk;
+  a->dv = dv;
+  a->dq_acc = reinterpret_cast<float*>(ws);
+  a->delta = reinterpret_cast<float*>(ws + round_up(rows * d * sizeof(float), 256));
+  a->lse2 = reinterpret_cast<float*>(ws + round_up(rows * d * sizeof(float), 256) +
+                                     round_up(padded * sizeof(float), 256));
+  a->B = B;
+  a->H = H;
+  a->N = N;
+  a->d = d;
+  a->causal = causal ? 1 : 0;
+  a->scale = scale;
+  a->status = di.status;
+  a->num_sms = di.num_sms;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal,
+           float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  fa::BwdArgs a;
+  int rc = bwd_prepare(kStagePre | kStageMain | kStageConvert, q, k, v, o, lse, dO, dq, dk, dv, B,
+                       H, N, d, causal, scale, workspace, workspace_bytes, &a);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = from_cuda(fa::launch_bwd_pre(a, st)))) return rc;
+  if ((rc = from_cuda(fa::launch_bwd_main(a, st)))) return rc;
+  return from_cuda(fa::launch_bwd_convert(a, st));
+}
+
+int fa_bwd_preprocess(const void* o, const float* lse, const void* dO, int B, int H, int N, int d,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  fa::BwdArgs a;
+  int rc = bwd_prepare(kStagePre, nullptr, nullptr, nullptr, o, lse, dO, nullptr, nullptr, nullptr,
+                       B, H, N, d, 0, 1.0f, workspace, workspace_bytes, &a);
+  if (rc) return rc;
+  return from_cuda(fa::launch_bwd_pre(a, static_cast<cudaStream_t>(stream)));
+}
+
+int fa_bwd_kv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+              int B, int H, int N, int d, int causal, float scale, void* workspace,
+              size_t workspace_bytes, void* stream) {
+  fa::BwdArgs a;
+  int rc = bwd_prepare(kStageMain, q, k, v, nullptr, nullptr, dO, nullptr, dk, dv, B, H, N, d,
+                       causal, scale, workspace, workspace_bytes, &a);
+  if (rc) return rc;
+  return from_cuda(fa::launch_bwd_main(a, static_cast<cudaStream_t>(stream)));
+}
+
+int fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  fa::BwdArgs a;
+  int rc = bwd_prepare(kStageConvert, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dq,
+                       nullptr, nullptr, B, H, N, d, 0, scale, workspace, workspace_bytes, &a);
+  if (rc) return rc;
+  return from_cuda(fa::launch_bwd_convert(a, static_cast<cudaStream_t>(stream)));
 }
 
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H,

@@ -463,57 +463,64 @@ __global__ void __launch_bounds__(256)
                  pack_bf16x2(y.x * scale, y.y * scale), pack_bf16x2(y.z * scale, y.w * scale));
 }
 
-template <int D, bool CAUSAL>
-static cudaError_t launch_t(const BwdArgs& a, cudaStream_t st) {
-  using C = Cfg<D>;
+template <int D>
+static cudaError_t launch_pre_t(const BwdArgs& a, cudaStream_t st) {
   const int n_pad = (a.N + 127) / 128 * 128;
   const size_t rows = static_cast<size_t>(a.B) * a.H * a.N;
-  float* lse2 = a.lse2;
+  constexpr int kRowsPerBlock = 256 / (D / 8);
+  const long long row_blocks = (static_cast<long long>(rows) + kRowsPerBlock - 1) / kRowsPerBlock;
+  const long long acc_vec4 = static_cast<long long>(rows) * D / 4;
+  const long long zero_blocks = std::min<long long>((acc_vec4 + 255) / 256, 8LL * a.num_sms);
+  const long long grid = row_blocks + zero_blocks;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  bwd_pre_kernel<D><<<static_cast<unsigned>(grid), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse,
+      a.delta, a.lse2, a.dq_acc, a.B, a.H, a.N, n_pad, acc_vec4, static_cast<int>(row_blocks));
+  return cudaGetLastError();
+}
 
-  // 1. preprocess
-  {
-    constexpr int kRowsPerBlock = 256 / (D / 8);
-    const long long row_blocks = (static_cast<long long>(rows) + kRowsPerBlock - 1) / kRowsPerBlock;
-    const long long acc_vec4 = static_cast<long long>(rows) * D / 4;
-    const long long zero_blocks = std::min<long long>((acc_vec4 + 255) / 256, 4LL * a.num_sms * 8);
-    const long long grid = row_blocks + zero_blocks;
-    if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    bwd_pre_kernel<D><<<static_cast<unsigned>(grid), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse,
-        a.delta, lse2, a.dq_acc, a.B, a.H, a.N, n_pad, acc_vec4, static_cast<int>(row_blocks));
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  // 2. main
-  {
-    auto kern = bwd_main_kernel<D, CAUSAL>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    const int num_kvtiles = (a.N + BM - 1) / BM;
-    const long long grid = static_cast<long long>(a.B) * a.H * num_kvtiles;
-    kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, st>>>(
-        a.tm_q, a.tm_k, a.tm_v, a.tm_do, lse2, a.delta, a.dq_acc,
-        static_cast<__nv_bfloat16*>(a.dk), static_cast<__nv_bfloat16*>(a.dv), a.B, a.H, a.N, n_pad,
-        a.scale, a.scale * kLog2e, num_kvtiles, a.status, kDefaultWaitTimeoutNs);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  // 3. dQ conversion
-  {
-    const long long threads = static_cast<long long>(rows) * (D / 8);
-    const long long grid = (threads + 255) / 256;
-    dq_convert_kernel<D><<<static_cast<unsigned>(grid), 256, 0, st>>>(
-        a.dq_acc, static_cast<__nv_bfloat16*>(a.dq), a.B, a.H, a.N, a.scale);
-    return cudaGetLastError();
-  }
+template <int D, bool CAUSAL>
+static cudaError_t launch_main_t(const BwdArgs& a, cudaStream_t st) {
+  using C = Cfg<D>;
+  const int n_pad = (a.N + 127) / 128 * 128;
+  auto kern = bwd_main_kernel<D, CAUSAL>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int num_kvtiles = (a.N + BM - 1) / BM;
+  const long long grid = static_cast<long long>(a.B) * a.H * num_kvtiles;
+  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, st>>>(
+      a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.lse2, a.delta, a.dq_acc,
+      static_cast<__nv_bfloat16*>(a.dk), static_cast<__nv_bfloat16*>(a.dv), a.B, a.H, a.N, n_pad,
+      a.scale, a.scale * kLog2e, num_kvtiles, a.status, kDefaultWaitTimeoutNs);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_convert_t(const BwdArgs& a, cudaStream_t st) {
+  const size_t rows = static_cast<size_t>(a.B) * a.H * a.N;
+  const long long threads = static_cast<long long>(rows) * (D / 8);
+  const long long grid = (threads + 255) / 256;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  dq_convert_kernel<D><<<static_cast<unsigned>(grid), 256, 0, st>>>(
+      a.dq_acc, static_cast<__nv_bfloat16*>(a.dq), a.B, a.H, a.N, a.scale);
+  return cudaGetLastError();
 }
 
 }  // namespace bwd
 
-cudaError_t launch_bwd_sm100(const BwdArgs& a, cudaStream_t s) {
-  if (a.d == 64) return a.causal ? bwd::launch_t<64, true>(a, s) : bwd::launch_t<64, false>(a, s);
-  return a.causal ? bwd::launch_t<128, true>(a, s) : bwd::launch_t<128, false>(a, s);
+cudaError_t launch_bwd_pre(const BwdArgs& a, cudaStream_t s) {
+  return a.d == 64 ? bwd::launch_pre_t<64>(a, s) : bwd::launch_pre_t<128>(a, s);
+}
+
+cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t s) {
+  if (a.d == 64)
+    return a.causal ? bwd::launch_main_t<64, true>(a, s) : bwd::launch_main_t<64, false>(a, s);
+  return a.causal ? bwd::launch_main_t<128, true>(a, s) : bwd::launch_main_t<128, false>(a, s);
+}
+
+cudaError_t launch_bwd_convert(const BwdArgs& a, cudaStream_t s) {
+  return a.d == 64 ? bwd::launch_convert_t<64>(a, s) : bwd::launch_convert_t<128>(a, s);
 }
 
 }  // namespace fa

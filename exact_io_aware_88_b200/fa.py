@@ -55,6 +55,12 @@ _lib.fa_bwd_workspace_bytes.argtypes = [_I, _I, _I, _I]
 _lib.fa_bwd_workspace_bytes.restype = _SZ
 _lib.fa_bwd.argtypes = [_P] * 9 + [_I, _I, _I, _I, _I, _F, _P, _SZ, _P]
 _lib.fa_bwd.restype = _I
+_lib.fa_bwd_preprocess.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]
+_lib.fa_bwd_preprocess.restype = _I
+_lib.fa_bwd_kv.argtypes = [_P] * 6 + [_I, _I, _I, _I, _I, _F, _P, _SZ, _P]
+_lib.fa_bwd_kv.restype = _I
+_lib.fa_bwd_dq_convert.argtypes = [_P, _I, _I, _I, _I, _F, _P, _SZ, _P]
+_lib.fa_bwd_dq_convert.restype = _I
 _lib.fa_fwd_f32.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.fa_fwd_f32.restype = _I
 _lib.fa_read_device_status.argtypes = [ctypes.POINTER(_I), _P]
@@ -69,8 +75,9 @@ _lib.fa_debug_wait_timeout.argtypes = [ctypes.c_longlong, _P]
 _lib.fa_debug_wait_timeout.restype = _I
 
 # Every symbol the C headers declare, for the ABI self-check.
-EXPORTED = ["fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_fwd_f32", "fa_read_device_status",
-            "fa_status_string", "fa_version", "fa_debug_umma_tile", "fa_debug_wait_timeout"]
+EXPORTED = sorted(["fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_kv",
+                   "fa_bwd_dq_convert", "fa_fwd_f32", "fa_read_device_status", "fa_status_string",
+                   "fa_version", "fa_debug_umma_tile", "fa_debug_wait_timeout"])
 
 
 def _ptr(x) -> Optional[int]:
@@ -111,6 +118,23 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, workspace
     return _lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
                        _ptr(dk), _ptr(dv), B, H, N, d, int(causal), float(scale),
                        _ptr(workspace), int(workspace_bytes), _stream(stream))
+
+
+def fa_bwd_preprocess(o, lse, dO, B, H, N, d, workspace, workspace_bytes, stream=None) -> int:
+    return _lib.fa_bwd_preprocess(_ptr(o), _ptr(lse), _ptr(dO), B, H, N, d, _ptr(workspace),
+                                  int(workspace_bytes), _stream(stream))
+
+
+def fa_bwd_kv(q, k, v, dO, dk, dv, B, H, N, d, causal, scale, workspace, workspace_bytes,
+              stream=None) -> int:
+    return _lib.fa_bwd_kv(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dk), _ptr(dv), B, H, N, d,
+                          int(causal), float(scale), _ptr(workspace), int(workspace_bytes),
+                          _stream(stream))
+
+
+def fa_bwd_dq_convert(dq, B, H, N, d, scale, workspace, workspace_bytes, stream=None) -> int:
+    return _lib.fa_bwd_dq_convert(_ptr(dq), B, H, N, d, float(scale), _ptr(workspace),
+                                  int(workspace_bytes), _stream(stream))
 
 
 def fa_fwd_f32(q, k, v, o, lse, B, H, N, d, causal, scale, stream=None) -> int:

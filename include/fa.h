@@ -79,6 +79,22 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            int B, int H, int N, int d, int causal, float scale,
            void* workspace, size_t workspace_bytes, void* stream);
 
+/* The three stages fa_bwd runs, exposed so a caller can time or schedule them apart.
+ * Calling them in this order on one stream with the same workspace is exactly fa_bwd.
+ *  fa_bwd_preprocess: D = rowsum(dO o O) and lse*log2(e) into the workspace; clears the
+ *                     workspace's fp32 dQ accumulator.  Reads o, lse, dO.
+ *  fa_bwd_kv:         the recompute kernel: per key/value tile, rebuilds S^T and P^T from
+ *                     the workspace statistics, writes dk, dv and adds dS K into the dQ
+ *                     accumulator.  Reads q, k, v, dO; needs fa_bwd_preprocess first.
+ *  fa_bwd_dq_convert: dq = bf16(scale * accumulator). */
+int fa_bwd_preprocess(const void* o, const float* lse, const void* dO, int B, int H, int N,
+                      int d, void* workspace, size_t workspace_bytes, void* stream);
+int fa_bwd_kv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+              int B, int H, int N, int d, int causal, float scale, void* workspace,
+              size_t workspace_bytes, void* stream);
+int fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
 /* Forward pass in fp32 on the CUDA cores (no tensor cores, no TF32), for fp32 inputs.
  *   q, k, v, o : [B][N][H][d] fp32; lse : [B][H][N] fp32.  1 <= d <= 128, d % 4 == 0. */
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
