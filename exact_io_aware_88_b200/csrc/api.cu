@@ -260,6 +260,57 @@ int fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, void* w
   return from_cuda(fa::launch_bwd_convert(a, static_cast<cudaStream_t>(stream)));
 }
 
+}  // extern "C"
+
+namespace {
+
+// Workspace of fa_bwd_noalloc: a fixed device array, one per GPU that loads the library.
+// Host code cannot use the symbol as a device address; its address is looked up once
+// per device (below) and handed to the kernels.
+static __device__ __align__(256) unsigned char g_noalloc_workspace[FA_NOALLOC_WORKSPACE_BYTES];
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_workspace on the current device (set-up on first use).
+int noalloc_workspace(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_workspace) != cudaSuccess || p == nullptr)
+      return FA_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                   int causal, float scale, void* stream) {
+  // Reject bad or oversized problems before touching the device.
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  int rc = check_shape(B, H, N, d, scale);
+  if (rc) return rc;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (fa_bwd_workspace_bytes(B, H, N, d) > FA_NOALLOC_WORKSPACE_BYTES) return FA_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if ((rc = noalloc_workspace(&ws))) return rc;
+  fa::BwdArgs a;
+  rc = bwd_prepare(kStagePre | kStageMain | kStageConvert, q, k, v, o, lse, dO, dq, dk, dv, B, H,
+                   N, d, causal, scale, ws, FA_NOALLOC_WORKSPACE_BYTES, &a);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = from_cuda(fa::launch_bwd_pre(a, st)))) return rc;
+  if ((rc = from_cuda(fa::launch_bwd_main(a, st)))) return rc;
+  return from_cuda(fa::launch_bwd_convert(a, st));
+}
+
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H,
                int N, int d, int causal, float scale, void* stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;

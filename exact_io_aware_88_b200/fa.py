@@ -61,6 +61,8 @@ _lib.fa_bwd_kv.argtypes = [_P] * 6 + [_I, _I, _I, _I, _I, _F, _P, _SZ, _P]
 _lib.fa_bwd_kv.restype = _I
 _lib.fa_bwd_dq_convert.argtypes = [_P, _I, _I, _I, _I, _F, _P, _SZ, _P]
 _lib.fa_bwd_dq_convert.restype = _I
+_lib.fa_bwd_noalloc.argtypes = [_P] * 9 + [_I, _I, _I, _I, _I, _F, _P]
+_lib.fa_bwd_noalloc.restype = _I
 _lib.fa_fwd_f32.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.fa_fwd_f32.restype = _I
 _lib.fa_read_device_status.argtypes = [ctypes.POINTER(_I), _P]
@@ -76,7 +78,7 @@ _lib.fa_debug_wait_timeout.restype = _I
 
 # Every symbol the C headers declare, for the ABI self-check.
 EXPORTED = sorted(["fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_kv",
-                   "fa_bwd_dq_convert", "fa_fwd_f32", "fa_read_device_status", "fa_status_string",
+                   "fa_bwd_dq_convert", "fa_bwd_noalloc", "fa_fwd_f32", "fa_read_device_status", "fa_status_string",
                    "fa_version", "fa_debug_umma_tile", "fa_debug_wait_timeout"])
 
 
@@ -135,6 +137,19 @@ def fa_bwd_kv(q, k, v, dO, dk, dv, B, H, N, d, causal, scale, workspace, workspa
 def fa_bwd_dq_convert(dq, B, H, N, d, scale, workspace, workspace_bytes, stream=None) -> int:
     return _lib.fa_bwd_dq_convert(_ptr(dq), B, H, N, d, float(scale), _ptr(workspace),
                                   int(workspace_bytes), _stream(stream))
+
+
+# Size of the library's built-in workspace used by fa_bwd_noalloc (FA_NOALLOC_WORKSPACE_BYTES).
+NOALLOC_WORKSPACE_BYTES = 64 * 1024 * 1024
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, stream=None) -> int:
+    """fa_bwd without a caller-provided workspace, for callers that may not allocate device
+    memory (see include/fa.h).  Calls whose GPU work overlaps share one library array and
+    race; serialise them."""
+    return _lib.fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                               _ptr(dk), _ptr(dv), B, H, N, d, int(causal), float(scale),
+                               _stream(stream))
 
 
 def fa_fwd_f32(q, k, v, o, lse, B, H, N, d, causal, scale, stream=None) -> int:

@@ -95,6 +95,31 @@ int fa_bwd_kv(const void* q, const void* k, const void* v, const void* dO, void*
 int fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, void* workspace,
                       size_t workspace_bytes, void* stream);
 
+/* Backward pass for callers that cannot allocate device memory.
+ *
+ * Who needs it: code that may not call cudaMalloc -- for example a plugin hosted by a
+ * framework that owns all device memory through its own allocator and forbids direct
+ * driver allocations, or a latency-critical loop that cannot afford cudaMalloc's implicit
+ * device-wide synchronisation -- and so cannot provide fa_bwd's workspace.  This entry
+ * point has no counterpart in the source pages; it is fa_bwd with the workspace taken from
+ * a fixed array inside the library instead of from the caller.
+ *
+ * Same arguments and results as fa_bwd minus the workspace.  The caller still owns and
+ * passes every input and output.  The library holds FA_NOALLOC_WORKSPACE_BYTES of device
+ * memory per GPU that loads it, for the life of the process; problems whose
+ * fa_bwd_workspace_bytes() exceeds that are rejected with FA_ERR_WORKSPACE before anything
+ * is launched.  Nothing here allocates or frees memory.
+ *  - The first call on a device looks up the array's device address (set-up, once per
+ *    device, with that device current); make that first call before any stream capture.
+ *  - Every call on a device shares the one array.  Calls whose work overlaps on the GPU
+ *    (e.g. on two streams without ordering between them) race on it and give wrong
+ *    results; serialise them.  Each call re-initialises what it needs (the dQ accumulator
+ *    is cleared), so leftovers of a previous call do not matter. */
+#define FA_NOALLOC_WORKSPACE_BYTES (64u * 1024u * 1024u)
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv,
+                   int B, int H, int N, int d, int causal, float scale, void* stream);
+
 /* Forward pass in fp32 on the CUDA cores (no tensor cores, no TF32), for fp32 inputs.
  *   q, k, v, o : [B][N][H][d] fp32; lse : [B][H][N] fp32.  1 <= d <= 128, d % 4 == 0. */
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
