@@ -20,8 +20,9 @@
 //                epilogue: dK_j*scale, dV_j -> bf16.
 //  3. dq_convert dq = bf16(scale * dQacc).                                     (HBM-bound)
 //
-// bwd_main CTA = 10 warps: 0-3 compute (thread t owns key row t = TMEM lane t), 4 TMA
-// producer, 5 TMEM allocator + MMA issuer, 6-9 dQ drain (thread owns query row = TMEM lane).
+// bwd_main CTA = 12 warps (3 warpgroups): 0-3 compute (thread t owns key row t = TMEM lane
+// t), 4-7 dQ drain (thread owns query row = TMEM lane), 8 TMA producer, 9 TMEM allocator +
+// MMA issuer, 10-11 idle.  setmaxnreg moves registers from the third warpgroup to compute.
 // TMEM (512 columns): dK [0,D), dV [D,2D), S^T/P^T [2D,2D+128), dP^T and then dQ
 // [2D+128,2D+256).
 #include <cuda.h>
@@ -39,7 +40,13 @@ namespace bwd {
 
 constexpr int BM = 128;  // key rows per CTA tile (MMA M)
 constexpr int BN = 128;  // query rows per step
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+// Registers per thread after the setmaxnreg split (launch gives 168 to each of the 384
+// threads = 64512): compute 240 + drain 168 + producer/MMA 72 = 480 per lane x 128 = 61440.
+constexpr uint32_t kRegsCompute = 240;
+constexpr uint32_t kRegsOther = 72;
+constexpr int kWarpLoad = 8;
+constexpr int kWarpMma = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -69,7 +76,7 @@ struct Bars {
   uint64_t kv_full;
   uint64_t q_full[2], q_empty[2];
   uint64_t do_full[2], do_empty[2];
-  uint64_t s_full, dp_full, ds_ready, dq_full, dq_empty, dkdv_done, drain;
+  uint64_t s_full, dp_full, p_ready, ds_ready, dq_full, dq_empty, dkdv_done, drain;
   uint32_t tmem_base;
   Abort abort;
 };
@@ -119,6 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
+    mbar_init(&bars->p_ready, 128);
     mbar_init(&bars->ds_ready, 128);
     mbar_init(&bars->dq_full, 1);
     mbar_init(&bars->dq_empty, 128);
@@ -127,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bars->abort.flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -145,115 +153,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* sVec = reinterpret_cast<float*>(smem + C::kOffVec);  // [stage][lse2 | D][128]
   const size_t vec_base = static_cast<size_t>(bh) * n_pad;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      prefetch_tmap(&tm_do);
-      const uint64_t pol_kv = policy_evict_first();
-      const uint64_t pol_q = policy_evict_last();
-      mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTileBytes);
-      for (int c = 0; c < C::kChunks; ++c) {
-        tma_load_4d(sK + c * C::kChunkBytes, &tm_k, &bars->kv_full, c * 64, h, k0, b, pol_kv);
-        tma_load_4d(sV + c * C::kChunkBytes, &tm_v, &bars->kv_full, c * 64, h, k0, b, pol_kv);
-      }
-      int issued_q = 0, issued_do = 0;
-      for (int n = 0; n < nq; ++n) {
-        const int i = i_begin + n;
-        const int sq = n % C::kQStages;
-        if (n >= C::kQStages &&
-            !mbar_wait(&bars->q_empty[sq], ((n / C::kQStages) - 1) & 1, ab, status, timeout_ns))
-          break;
-        mbar_arrive_expect_tx(&bars->q_full[sq], C::kTileBytes + 2 * BN * 4);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sQ + sq * C::kTileBytes + c * C::kChunkBytes, &tm_q, &bars->q_full[sq],
-                      c * 64, h, i * BN, b, pol_q);
-        bulk_load(sVec + sq * 2 * BN, lse2 + vec_base + i * BN, BN * 4, &bars->q_full[sq]);
-        bulk_load(sVec + sq * 2 * BN + BN, delta + vec_base + i * BN, BN * 4, &bars->q_full[sq]);
-        issued_q = n + 1;
-        const int sd = n % C::kDOStages;
-        if (n >= C::kDOStages &&
-            !mbar_wait(&bars->do_empty[sd], ((n / C::kDOStages) - 1) & 1, ab, status, timeout_ns))
-          break;
-        mbar_arrive_expect_tx(&bars->do_full[sd], C::kTileBytes);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sDO + sd * C::kTileBytes + c * C::kChunkBytes, &tm_do, &bars->do_full[sd],
-                      c * 64, h, i * BN, b, pol_q);
-        issued_do = n + 1;
-      }
-      // Drain every copy into shared memory before the CTA may exit.
-      Abort local{0};
-      mbar_wait(&bars->kv_full, 0, &local, status, timeout_ns);
-      for (int n = max(0, issued_q - C::kQStages); n < issued_q; ++n)
-        mbar_wait(&bars->q_full[n % C::kQStages], (n / C::kQStages) & 1, &local, status, timeout_ns);
-      for (int n = max(0, issued_do - C::kDOStages); n < issued_do; ++n)
-        mbar_wait(&bars->do_full[n % C::kDOStages], (n / C::kDOStages) & 1, &local, status,
-                  timeout_ns);
-    }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t id_sdp = idesc_bf16_f32(BM, BN, 0, 0);  // K_j Q_i^T, V_j dO_i^T
-      constexpr uint32_t id_dkdv = idesc_bf16_f32(BM, D, 0, 1);  // P^T dO_i, dS^T Q_i
-      constexpr uint32_t id_dq = idesc_bf16_f32(BN, D, 1, 1);    // dS K_j (A MN-major)
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ),
-                     aDO = smem_u32(sDO), aDS = smem_u32(sDS);
-      bool ok = mbar_wait(&bars->kv_full, 0, ab, status, timeout_ns);
-      for (int n = 0; ok && n < nq; ++n) {
-        const int sq = n % C::kQStages, sd = n % C::kDOStages;
-        if (!mbar_wait(&bars->q_full[sq], (n / C::kQStages) & 1, ab, status, timeout_ns)) break;
-        tc_fence_after();
-        const uint32_t qb = aQ + sq * C::kTileBytes, dob = aDO + sd * C::kTileBytes;
-        // S^T = K_j Q_i^T  (both K-major over the head dim)
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-          umma_ss(tbase + C::kColS, sdesc_sw128(aK + off, 16, 1024), sdesc_sw128(qb + off, 16, 1024),
-                  id_sdp, kk > 0);
-        }
-        umma_commit(&bars->s_full);
-        if (!mbar_wait(&bars->do_full[sd], (n / C::kDOStages) & 1, ab, status, timeout_ns)) break;
-        if (n > 0 && !mbar_wait(&bars->dq_empty, (n - 1) & 1, ab, status, timeout_ns)) break;
-        tc_fence_after();
-        // dP^T = V_j dO_i^T  (columns previously holding dQ_{i-1}, now drained)
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-          umma_ss(tbase + C::kColDP, sdesc_sw128(aV + off, 16, 1024),
-                  sdesc_sw128(dob + off, 16, 1024), id_sdp, kk > 0);
-        }
-        umma_commit(&bars->dp_full);
-        if (!mbar_wait(&bars->ds_ready, n & 1, ab, status, timeout_ns)) break;
-        tc_fence_after();
-        // dV_j += P^T dO_i   (A = P^T from TMEM, B = dO_i MN-major over the query index)
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts(tbase + C::kColDV, tbase + C::kColS + kk * 8,
-                  sdesc_sw128(dob + kk * 2048, C::kChunkBytes, 1024), id_dkdv, (n > 0 || kk > 0));
-        umma_commit(&bars->do_empty[sd]);
-        // dK_j += dS^T Q_i   (A = dS^T K-major over the query index, B = Q_i MN-major)
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-          umma_ss(tbase + C::kColDK, sdesc_sw128(aDS + aoff, 16, 1024),
-                  sdesc_sw128(qb + kk * 2048, C::kChunkBytes, 1024), id_dkdv, (n > 0 || kk > 0));
-        }
-        // dQ_i = dS K_j   (A = dS: the same smem tile read MN-major; B = K_j MN-major)
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ss(tbase + C::kColDP, sdesc_sw128(aDS + kk * 2048, C::kChunkBytes, 1024),
-                  sdesc_sw128(aK + kk * 2048, C::kChunkBytes, 1024), id_dq, kk > 0);
-        umma_commit(&bars->dq_full);
-        umma_commit(&bars->q_empty[sq]);
-      }
-      umma_commit(&bars->dkdv_done);
-      umma_commit(&bars->drain);
-      Abort local{0};
-      mbar_wait(&bars->drain, 0, &local, status, timeout_ns);
-    }
-  } else if (warp < 4) {
+  // Role dispatch by warpgroup, so that each warpgroup executes its register
+  // reallocation once, at one place, before its role's code.
+  if (warp < 4) {
+    regs_inc<kRegsCompute>();
     // ------------------------------------------------------------------ compute warps
     const int t = threadIdx.x;  // key row within the tile == TMEM lane
     const int key = k0 + t;
@@ -270,42 +173,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->q_full[sq], (n / C::kQStages) & 1, ab, status,
                                              timeout_ns));
       if (!ok) break;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, n & 1, ab, status, timeout_ns));
-      if (!ok) break;
       tc_fence_after();
+      // Phase 1: P^T = exp2(S^T * scale*log2e - lse2) -> bf16 into the S^T columns.
       // Columns c with q0 + c < key are masked (query before key) on diagonal tiles; keys
       // and queries past N are masked on tail tiles.
       const bool row_dead = key >= N;
       const int first_vis = CAUSAL ? key - q0 : 0;  // first visible column
       const int last_vis = N - 1 - q0;               // last existing column
+      float p[BN];
+#pragma unroll
+      for (int h32 = 0; h32 < 4; ++h32) {
+        uint32_t su[32];
+        tmem_ld32(lane_base + C::kColS + 32 * h32, su);
+#pragma unroll
+        for (int e4 = 0; e4 < 32; e4 += 4) {
+          const int c = 32 * h32 + e4;
+          const float4 l4 = *reinterpret_cast<const float4*>(sL + c);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float e = ex2_approx(fmaf(__uint_as_float(su[e4 + u]), scale_log2, -lv[u]));
+            p[c + u] = (row_dead || c + u < first_vis || c + u > last_vis) ? 0.f : e;
+          }
+        }
+      }
+#pragma unroll
+      for (int h32 = 0; h32 < 2; ++h32) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(p[64 * h32 + 2 * e], p[64 * h32 + 2 * e + 1]);
+        tmem_st32(lane_base + C::kColS + 32 * h32, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->p_ready);
+      // Phase 2: dS^T = P^T o (dP^T - D) -> bf16 into shared memory (swizzled rows).
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, n & 1, ab, status, timeout_ns));
+      if (!ok) break;
+      tc_fence_after();
 #pragma unroll
       for (int qq = 0; qq < 4; ++qq) {  // 32 query columns at a time
-        uint32_t su[32], du[32];
-        tmem_ld32(lane_base + C::kColS + qq * 32, su);
+        uint32_t du[32];
         tmem_ld32(lane_base + C::kColDP + qq * 32, du);
-        uint32_t ppk[16], dpk[16];
+        uint32_t dpk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const int c = qq * 32 + e;
-          const float4 l4 = *reinterpret_cast<const float4*>(sL + c);
           const float4 d4 = *reinterpret_cast<const float4*>(sD + c);
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-          const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-          float p[4], ds[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            p[u] = ex2_approx(fmaf(__uint_as_float(su[e + u]), scale_log2, -lv[u]));
-            if (row_dead || c + u < first_vis || c + u > last_vis) p[u] = 0.f;
-            ds[u] = p[u] * (__uint_as_float(du[e + u]) - dv4[u]);
-          }
-          ppk[e / 2] = pack_bf16x2(p[0], p[1]);
-          ppk[e / 2 + 1] = pack_bf16x2(p[2], p[3]);
-          dpk[e / 2] = pack_bf16x2(ds[0], ds[1]);
-          dpk[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+          dpk[e / 2] = pack_bf16x2(p[c] * (__uint_as_float(du[e]) - d4.x),
+                                   p[c + 1] * (__uint_as_float(du[e + 1]) - d4.y));
+          dpk[e / 2 + 1] = pack_bf16x2(p[c + 2] * (__uint_as_float(du[e + 2]) - d4.z),
+                                       p[c + 3] * (__uint_as_float(du[e + 3]) - d4.w));
         }
-        // P^T (bf16 pairs) into columns [16qq, 16qq+16) of the S^T region, whose S^T values
-        // were consumed by this or an earlier quarter.
-        tmem_st16(lane_base + C::kColS + qq * 16, ppk);
         // dS^T row t, query columns [32qq, 32qq+32): chunk qq/2, 16-byte pieces 4(qq%2)..+3.
         uint8_t* chunk = sDS + (qq >> 1) * C::kChunkBytes;
 #pragma unroll
@@ -313,7 +232,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(chunk + sw128_offset(t, (qq & 1) * 4 + pc)) =
               make_uint4(dpk[4 * pc], dpk[4 * pc + 1], dpk[4 * pc + 2], dpk[4 * pc + 3]);
       }
-      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars->ds_ready);
@@ -345,8 +263,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------------ dQ drain warps
+    // Load the whole dQ_i tile row into registers, hand the TMEM columns back at once, then
+    // reduce into the fp32 accumulator while the next tile's MMAs run.
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;  // query row within the tile
     const uint32_t lane_base = tbase + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -355,28 +275,159 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_full, n & 1, ab, status, timeout_ns));
       if (!ok) break;
       tc_fence_after();
-      float* dst = dq_acc + (static_cast<size_t>(bh) * N + q) * D;
+      uint32_t u[D];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld32(lane_base + C::kColDP + c * 32, u);
-        if (q < N) {
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            atomicAdd(reinterpret_cast<float4*>(dst + c * 32 + 4 * v),
-                      make_float4(__uint_as_float(u[4 * v]), __uint_as_float(u[4 * v + 1]),
-                                  __uint_as_float(u[4 * v + 2]), __uint_as_float(u[4 * v + 3])));
-        }
-      }
+      for (int c = 0; c < D / 64; ++c)
+        tmem_ld64(lane_base + C::kColDP + 64 * c, *reinterpret_cast<uint32_t(*)[64]>(&u[64 * c]));
       tc_fence_before();
       mbar_arrive(&bars->dq_empty);
+      if (q < N) {
+        float* dst = dq_acc + (static_cast<size_t>(bh) * N + q) * D;
+#pragma unroll
+        for (int v = 0; v < D / 4; ++v)
+          atomicAdd(reinterpret_cast<float4*>(dst + 4 * v),
+                    make_float4(__uint_as_float(u[4 * v]), __uint_as_float(u[4 * v + 1]),
+                                __uint_as_float(u[4 * v + 2]), __uint_as_float(u[4 * v + 3])));
+      }
+    }
+  } else {
+    regs_dec<kRegsOther>();
+    if (warp == kWarpLoad) {
+      // ------------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_do);
+        const uint64_t pol_kv = policy_evict_first();
+        const uint64_t pol_q = policy_evict_last();
+        mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTileBytes);
+        for (int c = 0; c < C::kChunks; ++c) {
+          tma_load_4d(sK + c * C::kChunkBytes, &tm_k, &bars->kv_full, c * 64, h, k0, b, pol_kv);
+          tma_load_4d(sV + c * C::kChunkBytes, &tm_v, &bars->kv_full, c * 64, h, k0, b, pol_kv);
+        }
+        int issued_q = 0, issued_do = 0;
+        for (int n = 0; n < nq; ++n) {
+          const int i = i_begin + n;
+          const int sq = n % C::kQStages;
+          if (n >= C::kQStages &&
+              !mbar_wait(&bars->q_empty[sq], ((n / C::kQStages) - 1) & 1, ab, status, timeout_ns))
+            break;
+          mbar_arrive_expect_tx(&bars->q_full[sq], C::kTileBytes + 2 * BN * 4);
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(sQ + sq * C::kTileBytes + c * C::kChunkBytes, &tm_q, &bars->q_full[sq],
+                        c * 64, h, i * BN, b, pol_q);
+          bulk_load(sVec + sq * 2 * BN, lse2 + vec_base + i * BN, BN * 4, &bars->q_full[sq]);
+          bulk_load(sVec + sq * 2 * BN + BN, delta + vec_base + i * BN, BN * 4, &bars->q_full[sq]);
+          issued_q = n + 1;
+          const int sd = n % C::kDOStages;
+          if (n >= C::kDOStages &&
+              !mbar_wait(&bars->do_empty[sd], ((n / C::kDOStages) - 1) & 1, ab, status, timeout_ns))
+            break;
+          mbar_arrive_expect_tx(&bars->do_full[sd], C::kTileBytes);
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(sDO + sd * C::kTileBytes + c * C::kChunkBytes, &tm_do, &bars->do_full[sd],
+                        c * 64, h, i * BN, b, pol_q);
+          issued_do = n + 1;
+        }
+        // Drain every copy into shared memory before the CTA may exit.
+        Abort local{0};
+        mbar_wait(&bars->kv_full, 0, &local, status, timeout_ns);
+        for (int n = max(0, issued_q - C::kQStages); n < issued_q; ++n)
+          mbar_wait(&bars->q_full[n % C::kQStages], (n / C::kQStages) & 1, &local, status, timeout_ns);
+        for (int n = max(0, issued_do - C::kDOStages); n < issued_do; ++n)
+          mbar_wait(&bars->do_full[n % C::kDOStages], (n / C::kDOStages) & 1, &local, status,
+                    timeout_ns);
+      }
+    } else if (warp == kWarpMma) {
+      // ------------------------------------------------------------------ MMA issuer
+      // Per query tile n (rows i = i_begin + n), in issue order:
+      //   [p_ready n]  dV += P^T_n dO_n                 -> releases dO_n
+      //                S^T_{n+1} = K Q_{n+1}^T (R1)      (P^T_n already consumed, in order)
+      //   [ds_ready n] dK += dS^T_n Q_n ; dQ_n = dS_n K (R2) -> releases Q_n
+      //   [dq_empty n] dP^T_{n+1} = V dO_{n+1}^T (R2)
+      // so the next S^T and dV overlap the dS computation, and the dQ drain only gates dP.
+      if (lane == 0) {
+        constexpr uint32_t id_sdp = idesc_bf16_f32(BM, BN, 0, 0);  // K_j Q_i^T, V_j dO_i^T
+        constexpr uint32_t id_dkdv = idesc_bf16_f32(BM, D, 0, 1);  // P^T dO_i, dS^T Q_i
+        constexpr uint32_t id_dq = idesc_bf16_f32(BN, D, 1, 1);    // dS K_j (A MN-major)
+        const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ),
+                       aDO = smem_u32(sDO), aDS = smem_u32(sDS);
+        auto issue_s = [&](int n) -> bool {  // S^T_n = K_j Q_n^T (K-major over the head dim)
+          const int sq = n % C::kQStages;
+          if (!mbar_wait(&bars->q_full[sq], (n / C::kQStages) & 1, ab, status, timeout_ns))
+            return false;
+          tc_fence_after();
+          const uint32_t qb = aQ + sq * C::kTileBytes;
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+            umma_ss(tbase + C::kColS, sdesc_sw128(aK + off, 16, 1024),
+                    sdesc_sw128(qb + off, 16, 1024), id_sdp, kk > 0);
+          }
+          umma_commit(&bars->s_full);
+          return true;
+        };
+        auto issue_dp = [&](int n) -> bool {  // dP^T_n = V_j dO_n^T
+          const int sd = n % C::kDOStages;
+          if (!mbar_wait(&bars->do_full[sd], (n / C::kDOStages) & 1, ab, status, timeout_ns))
+            return false;
+          if (n > 0 && !mbar_wait(&bars->dq_empty, (n - 1) & 1, ab, status, timeout_ns))
+            return false;
+          tc_fence_after();
+          const uint32_t dob = aDO + sd * C::kTileBytes;
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+            umma_ss(tbase + C::kColDP, sdesc_sw128(aV + off, 16, 1024),
+                    sdesc_sw128(dob + off, 16, 1024), id_sdp, kk > 0);
+          }
+          umma_commit(&bars->dp_full);
+          return true;
+        };
+        bool ok = mbar_wait(&bars->kv_full, 0, ab, status, timeout_ns) && issue_s(0) && issue_dp(0);
+        for (int n = 0; ok && n < nq; ++n) {
+          const int sq = n % C::kQStages, sd = n % C::kDOStages;
+          const uint32_t qb = aQ + sq * C::kTileBytes, dob = aDO + sd * C::kTileBytes;
+          if (!mbar_wait(&bars->p_ready, n & 1, ab, status, timeout_ns)) break;
+          tc_fence_after();
+          // dV_j += P^T dO_i   (A = P^T from TMEM, B = dO_i MN-major over the query index)
+  #pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            umma_ts(tbase + C::kColDV, tbase + C::kColS + kk * 8,
+                    sdesc_sw128(dob + kk * 2048, C::kChunkBytes, 1024), id_dkdv, (n > 0 || kk > 0));
+          umma_commit(&bars->do_empty[sd]);
+          if (n + 1 < nq && !issue_s(n + 1)) break;
+          if (!mbar_wait(&bars->ds_ready, n & 1, ab, status, timeout_ns)) break;
+          tc_fence_after();
+          // dK_j += dS^T Q_i   (A = dS^T K-major over the query index, B = Q_i MN-major)
+  #pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint32_t aoff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+            umma_ss(tbase + C::kColDK, sdesc_sw128(aDS + aoff, 16, 1024),
+                    sdesc_sw128(qb + kk * 2048, C::kChunkBytes, 1024), id_dkdv, (n > 0 || kk > 0));
+          }
+          // dQ_i = dS K_j   (A = dS: the same smem tile read MN-major; B = K_j MN-major)
+  #pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            umma_ss(tbase + C::kColDP, sdesc_sw128(aDS + kk * 2048, C::kChunkBytes, 1024),
+                    sdesc_sw128(aK + kk * 2048, C::kChunkBytes, 1024), id_dq, kk > 0);
+          umma_commit(&bars->dq_full);
+          umma_commit(&bars->q_empty[sq]);
+          if (n + 1 < nq && !issue_dp(n + 1)) break;
+        }
+        umma_commit(&bars->dkdv_done);
+        umma_commit(&bars->drain);
+        Abort local{0};
+        mbar_wait(&bars->drain, 0, &local, status, timeout_ns);
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     __syncwarp();
     tmem_dealloc(tbase, kTmemCols);
   }
