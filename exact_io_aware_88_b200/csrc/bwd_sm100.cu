@@ -20,9 +20,10 @@
 //                epilogue: dK_j*scale, dV_j -> bf16.
 //  3. dq_convert dq = bf16(scale * dQacc).                                     (HBM-bound)
 //
-// bwd_main CTA = 12 warps (3 warpgroups): 0-3 compute (thread t owns key row t = TMEM lane
-// t), 4-7 dQ drain (thread owns query row = TMEM lane), 8 TMA producer, 9 TMEM allocator +
-// MMA issuer, 10-11 idle.  setmaxnreg moves registers from the third warpgroup to compute.
+// bwd_main CTA = 16 warps (4 warpgroups): 0-7 compute (two warpgroups, each owning half of
+// the 128 query columns of a step; thread t of a warpgroup owns key row t = TMEM lane t),
+// 8-11 dQ drain (thread owns query row = TMEM lane), 12 TMA producer, 13 TMEM allocator +
+// MMA issuer, 14-15 idle.  setmaxnreg moves registers from the last warpgroup to the rest.
 // TMEM (512 columns): dK [0,D), dV [D,2D), S^T/P^T [2D,2D+128), dP^T and then dQ
 // [2D+128,2D+256).
 #include <cuda.h>
@@ -40,13 +41,18 @@ namespace bwd {
 
 constexpr int BM = 128;  // key rows per CTA tile (MMA M)
 constexpr int BN = 128;  // query rows per step
-constexpr int kThreads = 384;
-// Registers per thread after the setmaxnreg split (launch gives 168 to each of the 384
-// threads = 64512): compute 240 + drain 168 + producer/MMA 72 = 480 per lane x 128 = 61440.
-constexpr uint32_t kRegsCompute = 240;
+constexpr int kThreads = 512;
+// 16 warps = 4 warpgroups; sub-partition k runs warps k, k+4, k+8, k+12, one from each
+// warpgroup.  Launch gives 128 registers to every thread (65536); after setmaxnreg each
+// sub-partition holds 152 + 152 + 136 + 72 = 512 registers per lane (= 512 launched).
+constexpr uint32_t kRegsLaunch = 65536 / kThreads;  // 128 (ptxas allocates this at launch)
+constexpr uint32_t kRegsCompute = 152;
+constexpr uint32_t kRegsDrain = 136;
 constexpr uint32_t kRegsOther = 72;
-constexpr int kWarpLoad = 8;
-constexpr int kWarpMma = 9;
+static_assert(2 * kRegsCompute + kRegsDrain + kRegsOther <= 4 * kRegsLaunch,
+              "register split exceeds what the block is launched with");
+constexpr int kWarpLoad = 12;
+constexpr int kWarpMma = 13;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -56,7 +62,7 @@ struct Cfg {
   static constexpr int kChunkBytes = 128 * 128;  // one TMA box: 128 rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
   static constexpr int kQStages = 2;
-  static constexpr int kDOStages = (D == 128) ? 1 : 2;
+  static constexpr int kDOStages = 2;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kTileBytes;
   static constexpr int kOffQ = kOffV + kTileBytes;
@@ -65,7 +71,9 @@ struct Cfg {
   static constexpr int kOffVec = kOffDS + 2 * kChunkBytes;         // lse2 / D per q stage
   static constexpr int kVecBytes = kQStages * 2 * BN * 4;
   static constexpr int kOffBar = kOffVec + kVecBytes;
-  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+  // No alignment slack: the dynamic shared window starts 1024-byte aligned (checked at
+  // run time; a misaligned base makes the kernel report FA_ERR_UNSUPPORTED and return).
+  static constexpr int kSmemBytes = kOffBar + 256;
   static constexpr uint32_t kColDK = 0;
   static constexpr uint32_t kColDV = D;
   static constexpr uint32_t kColS = 2 * D;
@@ -89,6 +97,18 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// With head dim 128 the dQ tile is produced transposed (M = head dim), so that a warp's
+// fp32 reductions into the accumulator cover 128 contiguous bytes of one query row: one
+// L2 request per warp instruction instead of 32 scattered 16-byte pieces.  Head dim 64
+// keeps M = 128 query rows (an M = 64 accumulator has a different TMEM layout).
+template <int D>
+constexpr bool kDqTransposed = (D == 128);
+
+// TMEM column of the A operand (packed P^T) for K step kk of the dV product: compute
+// warpgroup h stores its 64 query columns as 32 packed columns at [64h, 64h+32) of the
+// S^T region, i.e. inside the S^T columns it has already read.
+__device__ __forceinline__ uint32_t p_col(int kk) { return 64u * (kk >> 2) + 8u * (kk & 3); }
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -99,9 +119,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float scale, float scale_log2, int num_kvtiles, int* status,
                     uint64_t timeout_ns) {
   using C = Cfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {  // 128-byte-swizzled tiles need a 1024-aligned base
+    if (threadIdx.x == 0) atomicCAS(status, FA_OK, FA_ERR_UNSUPPORTED);
+    return;
+  }
   Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -126,8 +148,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->p_ready, 128);
-    mbar_init(&bars->ds_ready, 128);
+    mbar_init(&bars->p_ready, 256);
+    mbar_init(&bars->ds_ready, 256);
     mbar_init(&bars->dq_full, 1);
     mbar_init(&bars->dq_empty, 128);
     mbar_init(&bars->dkdv_done, 1);
@@ -152,57 +174,60 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sDS = smem + C::kOffDS;
   float* sVec = reinterpret_cast<float*>(smem + C::kOffVec);  // [stage][lse2 | D][128]
   const size_t vec_base = static_cast<size_t>(bh) * n_pad;
+  const int wg = warp >> 2;
 
   // Role dispatch by warpgroup, so that each warpgroup executes its register
   // reallocation once, at one place, before its role's code.
-  if (warp < 4) {
-    regs_inc<kRegsCompute>();
+  if (wg < 2) {
+    regs_set<kRegsLaunch, kRegsCompute>();
     // ------------------------------------------------------------------ compute warps
-    const int t = threadIdx.x;  // key row within the tile == TMEM lane
+    // Warpgroup `half` handles query columns [64*half, 64*half+64) of every step for key
+    // row t (= TMEM lane t).
+    const int half = wg;
+    const int t = (warp & 3) * 32 + lane;
     const int key = k0 + t;
-    const uint32_t lane_base = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t lane_base = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t colS = C::kColS + 64 * half;
+    const uint32_t colDP = C::kColDP + 64 * half;
     bool ok = true;
     for (int n = 0; n < nq; ++n) {
       const int i = i_begin + n;
       const int q0 = i * BN;
       const int sq = n % C::kQStages;
-      const float* sL = sVec + sq * 2 * BN;
-      const float* sD = sL + BN;
+      const float4* gL = reinterpret_cast<const float4*>(sVec + sq * 2 * BN + 64 * half);
+      const float4* gD = reinterpret_cast<const float4*>(sVec + sq * 2 * BN + BN + 64 * half);
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, n & 1, ab, status, timeout_ns));
       if (!ok) break;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->q_full[sq], (n / C::kQStages) & 1, ab, status,
                                              timeout_ns));
       if (!ok) break;
       tc_fence_after();
-      // Phase 1: P^T = exp2(S^T * scale*log2e - lse2) -> bf16 into the S^T columns.
-      // Columns c with q0 + c < key are masked (query before key) on diagonal tiles; keys
-      // and queries past N are masked on tail tiles.
+      // Phase 1: P^T = exp2(S^T * scale*log2e - lse2) -> packed bf16 into TMEM.
+      // Column c (query q0 + c) is masked when it precedes the key (causal, diagonal
+      // tiles) or lies past N; key rows past N are masked whole.
       const bool row_dead = key >= N;
-      const int first_vis = CAUSAL ? key - q0 : 0;  // first visible column
-      const int last_vis = N - 1 - q0;               // last existing column
-      float p[BN];
+      const int first_vis = (CAUSAL ? key - q0 : 0) - 64 * half;  // in this half's columns
+      const int last_vis = N - 1 - q0 - 64 * half;
+      float p[64];
+      {
+        uint32_t su[64];
+        tmem_ld64(lane_base + colS, su);
 #pragma unroll
-      for (int h32 = 0; h32 < 4; ++h32) {
-        uint32_t su[32];
-        tmem_ld32(lane_base + C::kColS + 32 * h32, su);
-#pragma unroll
-        for (int e4 = 0; e4 < 32; e4 += 4) {
-          const int c = 32 * h32 + e4;
-          const float4 l4 = *reinterpret_cast<const float4*>(sL + c);
+        for (int c = 0; c < 64; c += 4) {
+          const float4 l4 = gL[c / 4];
           const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const float e = ex2_approx(fmaf(__uint_as_float(su[e4 + u]), scale_log2, -lv[u]));
+            const float e = ex2_approx(fmaf(__uint_as_float(su[c + u]), scale_log2, -lv[u]));
             p[c + u] = (row_dead || c + u < first_vis || c + u > last_vis) ? 0.f : e;
           }
         }
       }
-#pragma unroll
-      for (int h32 = 0; h32 < 2; ++h32) {
+      {
         uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(p[64 * h32 + 2 * e], p[64 * h32 + 2 * e + 1]);
-        tmem_st32(lane_base + C::kColS + 32 * h32, pk);
+        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
+        tmem_st32(lane_base + colS, pk);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -212,24 +237,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {  // 32 query columns at a time
+      for (int c32 = 0; c32 < 2; ++c32) {
         uint32_t du[32];
-        tmem_ld32(lane_base + C::kColDP + qq * 32, du);
+        tmem_ld32(lane_base + colDP + 32 * c32, du);
         uint32_t dpk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          const int c = qq * 32 + e;
-          const float4 d4 = *reinterpret_cast<const float4*>(sD + c);
+          const int c = 32 * c32 + e;
+          const float4 d4 = gD[c / 4];
           dpk[e / 2] = pack_bf16x2(p[c] * (__uint_as_float(du[e]) - d4.x),
                                    p[c + 1] * (__uint_as_float(du[e + 1]) - d4.y));
           dpk[e / 2 + 1] = pack_bf16x2(p[c + 2] * (__uint_as_float(du[e + 2]) - d4.z),
                                        p[c + 3] * (__uint_as_float(du[e + 3]) - d4.w));
         }
-        // dS^T row t, query columns [32qq, 32qq+32): chunk qq/2, 16-byte pieces 4(qq%2)..+3.
-        uint8_t* chunk = sDS + (qq >> 1) * C::kChunkBytes;
+        // dS^T row t, query columns [64*half + 32*c32, +32): chunk `half`, 16-byte pieces
+        // 4*c32 .. 4*c32+3.
+        uint8_t* chunk = sDS + half * C::kChunkBytes;
 #pragma unroll
         for (int pc = 0; pc < 4; ++pc)
-          *reinterpret_cast<uint4*>(chunk + sw128_offset(t, (qq & 1) * 4 + pc)) =
+          *reinterpret_cast<uint4*>(chunk + sw128_offset(t, 4 * c32 + pc)) =
               make_uint4(dpk[4 * pc], dpk[4 * pc + 1], dpk[4 * pc + 2], dpk[4 * pc + 3]);
       }
       fence_proxy_async_smem();
@@ -237,36 +263,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bars->ds_ready);
     }
     // ---------------------------------------------------------------- dK / dV epilogue
+    // Warpgroup 0 writes dK, warpgroup 1 writes dV.
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->dkdv_done, 0, ab, status, timeout_ns));
     if (ok) {
       tc_fence_after();
       const size_t orow = ((static_cast<size_t>(b) * N + key) * H + h) * D;
+      const uint32_t col = half == 0 ? C::kColDK : C::kColDV;
+      const float mul = half == 0 ? scale : 1.f;
+      __nv_bfloat16* dst = (half == 0 ? dk : dv) + orow;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t col = which == 0 ? C::kColDK : C::kColDV;
-        const float mul = which == 0 ? scale : 1.f;
-        __nv_bfloat16* dst = (which == 0 ? dk : dv) + orow;
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld32(lane_base + col + c * 32, u);
+        if (key < N) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t u[32];
-          tmem_ld32(lane_base + col + c * 32, u);
-          if (key < N) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              d4[v4] = make_uint4(
-                  pack_bf16x2(__uint_as_float(u[8 * v4 + 0]) * mul, __uint_as_float(u[8 * v4 + 1]) * mul),
-                  pack_bf16x2(__uint_as_float(u[8 * v4 + 2]) * mul, __uint_as_float(u[8 * v4 + 3]) * mul),
-                  pack_bf16x2(__uint_as_float(u[8 * v4 + 4]) * mul, __uint_as_float(u[8 * v4 + 5]) * mul),
-                  pack_bf16x2(__uint_as_float(u[8 * v4 + 6]) * mul, __uint_as_float(u[8 * v4 + 7]) * mul));
-          }
+          for (int v4 = 0; v4 < 4; ++v4)
+            d4[v4] = make_uint4(
+                pack_bf16x2(__uint_as_float(u[8 * v4 + 0]) * mul, __uint_as_float(u[8 * v4 + 1]) * mul),
+                pack_bf16x2(__uint_as_float(u[8 * v4 + 2]) * mul, __uint_as_float(u[8 * v4 + 3]) * mul),
+                pack_bf16x2(__uint_as_float(u[8 * v4 + 4]) * mul, __uint_as_float(u[8 * v4 + 5]) * mul),
+                pack_bf16x2(__uint_as_float(u[8 * v4 + 6]) * mul, __uint_as_float(u[8 * v4 + 7]) * mul));
         }
       }
     }
-  } else if (warp < 8) {
+  } else if (wg == 2) {
+    regs_set<kRegsLaunch, kRegsDrain>();
     // ------------------------------------------------------------------ dQ drain warps
-    // Load the whole dQ_i tile row into registers, hand the TMEM columns back at once, then
-    // reduce into the fp32 accumulator while the next tile's MMAs run.
+    // Copy the dQ_i tile out of TMEM, hand the columns back, then reduce into the fp32
+    // accumulator while the next tile's MMAs run.
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;  // query row within the tile
     const uint32_t lane_base = tbase + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -275,25 +300,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_full, n & 1, ab, status, timeout_ns));
       if (!ok) break;
       tc_fence_after();
-      uint32_t u[D];
+      if constexpr (kDqTransposed<D>) {
+        // Thread = head-dim index dd; 32 query columns at a time.  Lanes of a warp hold 32
+        // consecutive dd of one query row: each reduction is one 128-byte line.
+        // The whole tile row is loaded first so the TMEM columns go back before any
+        // reduction is issued.
+        const int dd = r;
+        const int q0 = (i_begin + n) * BN;
+        float* dst = dq_acc + (static_cast<size_t>(bh) * N + q0) * D + dd;
+        uint32_t u[BN];
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c)
-        tmem_ld64(lane_base + C::kColDP + 64 * c, *reinterpret_cast<uint32_t(*)[64]>(&u[64 * c]));
-      tc_fence_before();
-      mbar_arrive(&bars->dq_empty);
-      if (q < N) {
+        for (int c64 = 0; c64 < BN / 64; ++c64)
+          tmem_ld64(lane_base + C::kColDP + 64 * c64, *reinterpret_cast<uint32_t(*)[64]>(&u[64 * c64]));
+        tc_fence_before();
+        mbar_arrive(&bars->dq_empty);
+        const int cmax = min(BN, N - q0);  // query rows past N are dropped
+#pragma unroll
+        for (int e = 0; e < BN; ++e)
+          if (e < cmax) red_add_f32(dst + static_cast<size_t>(e) * D, __uint_as_float(u[e]));
+      } else {
+        // Thread = query row; 64 columns at a time; the TMEM columns are handed back after
+        // the last load, before the last batch of reductions.
         float* dst = dq_acc + (static_cast<size_t>(bh) * N + q) * D;
 #pragma unroll
-        for (int v = 0; v < D / 4; ++v)
-          atomicAdd(reinterpret_cast<float4*>(dst + 4 * v),
-                    make_float4(__uint_as_float(u[4 * v]), __uint_as_float(u[4 * v + 1]),
-                                __uint_as_float(u[4 * v + 2]), __uint_as_float(u[4 * v + 3])));
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t u[64];
+          tmem_ld64(lane_base + C::kColDP + 64 * c, u);
+          if (c == D / 64 - 1) {
+            tc_fence_before();
+            mbar_arrive(&bars->dq_empty);
+          }
+          if (q < N) {
+#pragma unroll
+            for (int v = 0; v < 16; ++v)
+              red_add_v4(dst + 64 * c + 4 * v, __uint_as_float(u[4 * v]), __uint_as_float(u[4 * v + 1]),
+                         __uint_as_float(u[4 * v + 2]), __uint_as_float(u[4 * v + 3]));
+          }
+        }
       }
     }
   } else {
-    regs_dec<kRegsOther>();
+    regs_set<kRegsLaunch, kRegsOther>();
     if (warp == kWarpLoad) {
-      // ------------------------------------------------------------------ TMA producer
+      // ---------------------------------------------------------------- TMA producer
       if (lane == 0) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
@@ -334,13 +383,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         Abort local{0};
         mbar_wait(&bars->kv_full, 0, &local, status, timeout_ns);
         for (int n = max(0, issued_q - C::kQStages); n < issued_q; ++n)
-          mbar_wait(&bars->q_full[n % C::kQStages], (n / C::kQStages) & 1, &local, status, timeout_ns);
+          mbar_wait(&bars->q_full[n % C::kQStages], (n / C::kQStages) & 1, &local, status,
+                    timeout_ns);
         for (int n = max(0, issued_do - C::kDOStages); n < issued_do; ++n)
           mbar_wait(&bars->do_full[n % C::kDOStages], (n / C::kDOStages) & 1, &local, status,
                     timeout_ns);
       }
     } else if (warp == kWarpMma) {
-      // ------------------------------------------------------------------ MMA issuer
+      // ---------------------------------------------------------------- MMA issuer
       // Per query tile n (rows i = i_begin + n), in issue order:
       //   [p_ready n]  dV += P^T_n dO_n                 -> releases dO_n
       //                S^T_{n+1} = K Q_{n+1}^T (R1)      (P^T_n already consumed, in order)
@@ -350,7 +400,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         constexpr uint32_t id_sdp = idesc_bf16_f32(BM, BN, 0, 0);  // K_j Q_i^T, V_j dO_i^T
         constexpr uint32_t id_dkdv = idesc_bf16_f32(BM, D, 0, 1);  // P^T dO_i, dS^T Q_i
-        constexpr uint32_t id_dq = idesc_bf16_f32(BN, D, 1, 1);    // dS K_j (A MN-major)
+        constexpr uint32_t id_dq = kDqTransposed<D>
+                                       ? idesc_bf16_f32(D, BN, 1, 1)   // K_j^T dS^T
+                                       : idesc_bf16_f32(BN, D, 1, 1);  // dS K_j
         const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ),
                        aDO = smem_u32(sDO), aDS = smem_u32(sDS);
         auto issue_s = [&](int n) -> bool {  // S^T_n = K_j Q_n^T (K-major over the head dim)
@@ -359,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             return false;
           tc_fence_after();
           const uint32_t qb = aQ + sq * C::kTileBytes;
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
             umma_ss(tbase + C::kColS, sdesc_sw128(aK + off, 16, 1024),
@@ -376,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             return false;
           tc_fence_after();
           const uint32_t dob = aDO + sd * C::kTileBytes;
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
             umma_ss(tbase + C::kColDP, sdesc_sw128(aV + off, 16, 1024),
@@ -392,26 +444,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&bars->p_ready, n & 1, ab, status, timeout_ns)) break;
           tc_fence_after();
           // dV_j += P^T dO_i   (A = P^T from TMEM, B = dO_i MN-major over the query index)
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
-            umma_ts(tbase + C::kColDV, tbase + C::kColS + kk * 8,
+            umma_ts(tbase + C::kColDV, tbase + C::kColS + p_col(kk),
                     sdesc_sw128(dob + kk * 2048, C::kChunkBytes, 1024), id_dkdv, (n > 0 || kk > 0));
           umma_commit(&bars->do_empty[sd]);
           if (n + 1 < nq && !issue_s(n + 1)) break;
           if (!mbar_wait(&bars->ds_ready, n & 1, ab, status, timeout_ns)) break;
           tc_fence_after();
           // dK_j += dS^T Q_i   (A = dS^T K-major over the query index, B = Q_i MN-major)
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
             const uint32_t aoff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
             umma_ss(tbase + C::kColDK, sdesc_sw128(aDS + aoff, 16, 1024),
                     sdesc_sw128(qb + kk * 2048, C::kChunkBytes, 1024), id_dkdv, (n > 0 || kk > 0));
           }
-          // dQ_i = dS K_j   (A = dS: the same smem tile read MN-major; B = K_j MN-major)
-  #pragma unroll
-          for (int kk = 0; kk < BM / 16; ++kk)
-            umma_ss(tbase + C::kColDP, sdesc_sw128(aDS + kk * 2048, C::kChunkBytes, 1024),
-                    sdesc_sw128(aK + kk * 2048, C::kChunkBytes, 1024), id_dq, kk > 0);
+          if constexpr (kDqTransposed<D>) {
+            // dQ_i^T = K_j^T dS^T   (A = K_j read MN-major over the head dim, B = dS^T
+            // MN-major over the query index): TMEM lane = head-dim index, column = query.
+#pragma unroll
+            for (int kk = 0; kk < BM / 16; ++kk)
+              umma_ss(tbase + C::kColDP, sdesc_sw128(aK + kk * 2048, C::kChunkBytes, 1024),
+                      sdesc_sw128(aDS + kk * 2048, C::kChunkBytes, 1024), id_dq, kk > 0);
+          } else {
+            // dQ_i = dS K_j   (A = dS: the dS^T tile read MN-major; B = K_j MN-major)
+#pragma unroll
+            for (int kk = 0; kk < BM / 16; ++kk)
+              umma_ss(tbase + C::kColDP, sdesc_sw128(aDS + kk * 2048, C::kChunkBytes, 1024),
+                      sdesc_sw128(aK + kk * 2048, C::kChunkBytes, 1024), id_dq, kk > 0);
+          }
           umma_commit(&bars->dq_full);
           umma_commit(&bars->q_empty[sq]);
           if (n + 1 < nq && !issue_dp(n + 1)) break;

@@ -289,6 +289,17 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
       : "memory");
 }
 
+// Fire-and-forget fp32 vector reduction into global memory (no return value).
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ void red_add_f32(float* addr, float a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
+}
+
 // ----------------------------------------------------------------------------- registers
 
 // Warpgroup-wide register reallocation (all 128 threads of a warpgroup execute it).  The
@@ -300,6 +311,19 @@ __device__ __forceinline__ void regs_inc() {
 template <uint32_t kRegs>
 __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
+// Moves the calling warpgroup from the per-thread register count the kernel was launched
+// with (kLaunch, what ptxas allocates for the launch bounds) to kTarget: an increase must
+// use .inc and a decrease .dec, and the count must be a multiple of 8 in [24, 256].
+template <uint32_t kLaunch, uint32_t kTarget>
+__device__ __forceinline__ void regs_set() {
+  static_assert(kTarget % 8 == 0 && kTarget >= 24 && kTarget <= 256, "bad register count");
+  if constexpr (kTarget > kLaunch) {
+    regs_inc<kTarget>();
+  } else if constexpr (kTarget < kLaunch) {
+    regs_dec<kTarget>();
+  }
 }
 
 // ----------------------------------------------------------------------------- math
