@@ -596,8 +596,13 @@ static cudaError_t launch_main_t(const BwdArgs& a, cudaStream_t st) {
   using C = Cfg<D>;
   const int n_pad = (a.N + 127) / 128 * 128;
   auto kern = bwd_main_kernel<D, CAUSAL>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  // The setmaxnreg split assumes the kernel launches with exactly kRegsLaunch registers per
+  // thread; with fewer, the increasing warpgroups could never be satisfied.
+  cudaFuncAttributes fa_attr;
+  cudaError_t e = cudaFuncGetAttributes(&fa_attr, kern);
+  if (e != cudaSuccess) return e;
+  if (fa_attr.numRegs != static_cast<int>(kRegsLaunch)) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int num_kvtiles = (a.N + BM - 1) / BM;
   const long long grid = static_cast<long long>(a.B) * a.H * num_kvtiles;

@@ -1,26 +1,36 @@
-// fwd_sm100.cu -- attention forward on sm_100a: TMA K/V ring, tcgen05.mma into TMEM,
-// warp-specialised load / MMA / softmax warps, online softmax in base 2.
+// fwd_sm100.cu -- attention forward on sm_100a: persistent, warp-specialised, two query
+// tiles per CTA in ping-pong, TMA K/V ring, tcgen05.mma into TMEM, online softmax in base 2.
 //
 // The algorithm is the tiled, fused evaluation of softmax(scale*QK^T)V described in
 // "Flash Attention 2で打破するローカルLLMの「メモリの壁」" (section タイリング（Tiling）と
-// 再計算（Recomputation）の仕組み): a 128-row Q tile stays on chip while 128-row K/V tiles
-// stream past it; S and P live only in tensor memory.  The running max / sum rescaling that
+// 再計算（Recomputation）の仕組み): query tiles stay on chip while 128-row K/V tiles stream
+// past them; S and P live only in tensor memory.  The running max / sum rescaling that
 // keeps the softmax globally normalised is the one of "FlashAttention-2を読む" (section
 // タイル分割でも全体の正規化を保つ).  Non-matmul work is trimmed as in its first trick
 // (section GPUの稼働率を高める三つの工夫): the scale is folded into one FFMA before exp2,
 // masks are applied on diagonal / tail tiles only, 1/l is applied once at the end and the
 // output is rescaled only when a row's running max grows by more than 2^8 (exact: the final
-// normalisation uses the same, possibly stale, max).
+// normalisation uses the same, possibly stale, max).  Work is split along the sequence as
+// in its second trick: the persistent grid walks (batch*head, query-tile pair) units.
 //
-// CTA = 6 warps:
-//   warps 0-3  softmax: thread t owns query row t of the tile (= TMEM lane t)
-//   warp  4    TMA producer (one lane)
-//   warp  5    TMEM allocator + tcgen05.mma issuer (one lane)
-// TMEM (512 columns): S/P double buffer at columns [0,128) and [128,256); O at [256,256+D).
+// CTA = 12 warps (3 warpgroups):
+//   warps 0-3   softmax for query tile 0 of the pair (thread t owns row t = TMEM lane t)
+//   warps 4-7   softmax for query tile 1
+//   warp  8     TMA producer (one lane);  warp 9: TMEM allocator + tcgen05.mma issuer
+//   warps 10-11 idle
+// TMEM (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+//
+// Tensor-core issue order per K/V tile j (after S0(0), S1(0)):
+//   PV0(j), S0(j+1), PV1(j), S1(j+1)
+// so each tile's softmax runs while the tensor core works on the other tile, and by the
+// time softmax t sees S_t(j+1) the product PV_t(j) has completed (tcgen05 operations of
+// one thread complete in order), so O_t may be rescaled in place without another wait.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <algorithm>
 
 #include "launch.h"
 #include "ptx.cuh"
@@ -28,11 +38,18 @@
 namespace fa {
 namespace fwd {
 
-constexpr int BM = 128;               // query rows per tile
-constexpr int BN = 128;               // key rows per tile
-constexpr int kThreads = 192;
+constexpr int BM = 128;  // query rows per tile (two tiles per unit)
+constexpr int BN = 128;  // key rows per tile
+constexpr int kThreads = 384;
+// Launch gives 65536 / 384 -> 168 registers per thread; the softmax warpgroups take
+// registers from the producer / MMA warpgroup: 200 + 200 + 104 = 504 = 3 x 168.
+constexpr uint32_t kRegsLaunch = 168;
+constexpr uint32_t kRegsSoftmax = 200;
+constexpr uint32_t kRegsOther = 104;
+static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * kRegsLaunch, "register split too large");
+constexpr int kWarpLoad = 8;
+constexpr int kWarpMma = 9;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int D>
@@ -40,69 +57,94 @@ struct Cfg {
   static constexpr int kChunks = D / 64;              // 64-element (128-byte) column chunks
   static constexpr int kChunkBytes = BM * 128;        // one TMA box: 128 rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStages = (D == 128) ? 3 : 4;
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kTileBytes;
+  static constexpr int kStages = (D == 128) ? 2 : 4;  // K/V ring depth
+  static constexpr int kOffQ = 0;                     // Q0, Q1
+  static constexpr int kOffK = kOffQ + 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
+  static constexpr int kSmemBytes = kOffBar + 256;    // base is 1024-aligned (checked)
+  static constexpr uint32_t kColO = 256;
 };
 
 struct Bars {
-  uint64_t q_full;
-  uint64_t k_full[4];
-  uint64_t v_full[4];
-  uint64_t kv_empty[4];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t o_done;
+  uint64_t q_full, q_empty;
+  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+  uint64_t s_full[2], p_full[2], o_done[2], o_free[2];
   uint64_t drain;
   uint32_t tmem_base;
   Abort abort;
 };
 
+// Unit schedule shared by every role.  Round r hands CTA c the unit r*G + c (even r) or
+// r*G + G-1-c (odd r): a snake over the persistent grid.  Under the causal mask units are
+// sorted longest first (pair index descending), so each round is a band of similar cost
+// and the snake evens the per-CTA sums.
+struct Unit {
+  int bh, pair;
+};
+__device__ __forceinline__ int unit_of_round(int r, int G) {
+  const int c = static_cast<int>(blockIdx.x);
+  return r * G + ((r & 1) ? (G - 1 - c) : c);
+}
+template <bool CAUSAL>
+__device__ __forceinline__ Unit decode_unit(int u, int BH, int num_pairs) {
+  Unit x;
+  if (CAUSAL) {
+    x.pair = num_pairs - 1 - u / BH;
+    x.bh = u % BH;
+  } else {
+    x.bh = u / num_pairs;
+    x.pair = u % num_pairs;
+  }
+  return x;
+}
+
+// K/V tiles visible to query tile t (0 or 1) of pair p.
+template <bool CAUSAL>
+__device__ __forceinline__ int kv_tiles(int pair, int t, int kv_total) {
+  return CAUSAL ? min(kv_total, 2 * pair + t + 1) : kv_total;
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
-               float* __restrict__ lse, int B, int H, int N, float scale_log2, int num_qtiles,
+               float* __restrict__ lse, int B, int H, int N, float scale_log2, int num_pairs,
                int* status, uint64_t timeout_ns) {
   using C = Cfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {  // 128-byte-swizzled tiles need a 1024-aligned base
+    if (threadIdx.x == 0) atomicCAS(status, FA_OK, FA_ERR_UNSUPPORTED);
+    return;
+  }
   Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // Work unit: (b, h) major so that concurrently running CTAs share K/V in L2; within a
-  // head, causal tiles run longest first.
-  const int bh = blockIdx.x / num_qtiles;
-  int qt = blockIdx.x % num_qtiles;
-  if (CAUSAL) qt = num_qtiles - 1 - qt;
-  const int b = bh / H, h = bh % H;
-  const int q0 = qt * BM;
-  const int kv_tiles_total = (N + BN - 1) / BN;
-  const int nkv = CAUSAL ? min(kv_tiles_total, qt + 1) : kv_tiles_total;
+  const int BH = B * H;
+  const int num_units = BH * num_pairs;
+  const int G = gridDim.x;
+  const int kv_total = (N + BN - 1) / BN;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], BM);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_full[t], BM);
+      mbar_init(&bars->o_done[t], 1);
+      mbar_init(&bars->o_free[t], BM);
     }
-    mbar_init(&bars->o_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort.flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -111,208 +153,289 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = bars->tmem_base;
   Abort* ab = &bars->abort;
-
   uint8_t* sQ = smem + C::kOffQ;
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
+  const int wg = warp >> 2;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      const uint64_t pol_q = policy_evict_first();
-      const uint64_t pol_kv = policy_evict_last();
-      mbar_arrive_expect_tx(&bars->q_full, C::kTileBytes);
-      for (int c = 0; c < C::kChunks; ++c)
-        tma_load_4d(sQ + c * C::kChunkBytes, &tm_q, &bars->q_full, c * 64, h, q0, b, pol_q);
-      int issued = 0;
-      for (int j = 0; j < nkv; ++j) {
-        const int s = j % C::kStages;
-        if (j >= C::kStages &&
-            !mbar_wait(&bars->kv_empty[s], ((j / C::kStages) - 1) & 1, ab, status, timeout_ns))
-          break;
-        uint8_t* dk = sK + s * C::kTileBytes;
-        uint8_t* dv = sV + s * C::kTileBytes;
-        mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(dk + c * C::kChunkBytes, &tm_k, &bars->k_full[s], c * 64, h, j * BN, b,
-                      pol_kv);
-        mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(dv + c * C::kChunkBytes, &tm_v, &bars->v_full[s], c * 64, h, j * BN, b,
-                      pol_kv);
-        issued = j + 1;
-      }
-      // Drain: make sure no copy into this CTA's shared memory is still in flight.
-      uint32_t drained = 1;
-      Abort local{0};
-      drained &= mbar_wait(&bars->q_full, 0, &local, status, timeout_ns);
-      for (int j = (issued > C::kStages ? issued - C::kStages : 0); j < issued; ++j) {
-        const int s = j % C::kStages;
-        drained &= mbar_wait(&bars->k_full[s], (j / C::kStages) & 1, &local, status, timeout_ns);
-        drained &= mbar_wait(&bars->v_full[s], (j / C::kStages) & 1, &local, status, timeout_ns);
-      }
-      (void)drained;
-    }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(BM, D, 0, 1);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-      bool ok = mbar_wait(&bars->q_full, 0, ab, status, timeout_ns);
-      tc_fence_after();
-      auto issue_s = [&](int j) -> bool {
-        const int s = j % C::kStages;
-        if (!mbar_wait(&bars->k_full[s], (j / C::kStages) & 1, ab, status, timeout_ns))
-          return false;
-        tc_fence_after();
-        const uint32_t d_tmem = tbase + (j & 1) * BN;
-        const uint32_t kbase = aK + s * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-          umma_ss(d_tmem, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
-                  idesc_s, kk > 0);
-        }
-        umma_commit(&bars->s_full[j & 1]);
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; ok && j < nkv; ++j) {
-        if (j + 1 < nkv && !issue_s(j + 1)) break;
-        const int s = j % C::kStages;
-        if (!mbar_wait(&bars->p_full[j & 1], (j >> 1) & 1, ab, status, timeout_ns)) break;
-        if (!mbar_wait(&bars->v_full[s], (j / C::kStages) & 1, ab, status, timeout_ns)) break;
-        tc_fence_after();
-        const uint32_t vbase = aV + s * C::kTileBytes;
-        const uint32_t p_tmem = tbase + (j & 1) * BN;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          umma_ts(tbase + kColO, p_tmem + kk * 8, sdesc_sw128(vbase + kk * 2048, C::kChunkBytes, 1024),
-                  idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&bars->kv_empty[s]);
-        umma_commit(&bars->o_done);
-      }
-      // Drain every MMA this thread issued before TMEM is released.
-      umma_commit(&bars->drain);
-      Abort local{0};
-      mbar_wait(&bars->drain, 0, &local, status, timeout_ns);
-    }
-  } else {
+  // Role dispatch by warpgroup: each warpgroup reallocates its registers once, up front.
+  if (wg < 2) {
+    regs_set<kRegsLaunch, kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax warps
-    const int r = threadIdx.x;  // row within the tile == TMEM lane
-    const int row = q0 + r;
-    const uint32_t lane_base = tbase + (static_cast<uint32_t>(warp * 32) << 16);
-    float m = -INFINITY;  // running max of scale*log2(e)*s (possibly stale by < 2^8)
-    float l = 0.f;
+    const int t = wg;                      // query tile of the pair
+    const int r = (warp & 3) * 32 + lane;  // row within the tile == TMEM lane
+    const uint32_t lane_base = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t colS = BN * t;
+    const uint32_t colO = C::kColO + D * t;
+    int ns = 0;     // s_full phases consumed
+    int units = 0;  // units finished
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      // Every decision that guards a warp-collective tcgen05.ld/st is made warp-uniform.
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, ab, status,
-                                             timeout_ns));
+    for (int rr = 0; ok; ++rr) {
+      const int u = unit_of_round(rr, G);
+      if (u >= num_units) break;
+      const Unit x = decode_unit<CAUSAL>(u, BH, num_pairs);
+      const int b = x.bh / H, h = x.bh % H;
+      const int q0 = (2 * x.pair + t) * BM;
+      const int row = q0 + r;
+      const int nkv = kv_tiles<CAUSAL>(x.pair, t, kv_total);
+      float m = -INFINITY;  // running max of scale*log2(e)*s (possibly stale by < 2^8)
+      float l = 0.f;
+      for (int j = 0; j < nkv; ++j) {
+        // Decisions guarding warp-collective tcgen05.ld/st are made warp-uniform.
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], ns & 1, ab, status, timeout_ns));
+        if (!ok) break;
+        ++ns;
+        tc_fence_after();
+        float sv[BN];
+        {
+          uint32_t u0[64];
+          tmem_ld64(lane_base + colS, u0);
+#pragma unroll
+          for (int i = 0; i < 64; ++i) sv[i] = __uint_as_float(u0[i]);
+        }
+        {
+          uint32_t u1[64];
+          tmem_ld64(lane_base + colS + 64, u1);
+#pragma unroll
+          for (int i = 0; i < 64; ++i) sv[64 + i] = __uint_as_float(u1[i]);
+        }
+        const int k0 = j * BN;
+        if ((CAUSAL && k0 + BN - 1 > q0) || k0 + BN > N) {  // diagonal or tail tile
+          const int lim = min(CAUSAL ? row : N - 1, N - 1) - k0;  // last visible column
+#pragma unroll
+          for (int i = 0; i < BN; ++i)
+            if (i > lim) sv[i] = -INFINITY;
+        }
+        float mx = sv[0];
+#pragma unroll
+        for (int i = 1; i < BN; ++i) mx = fmaxf(mx, sv[i]);
+        const float m_tile = mx * scale_log2;
+        float alpha = 1.f;
+        bool need = false;
+        if (m == -INFINITY) {
+          m = m_tile;
+        } else if (m_tile - m > kRescaleThreshold) {
+          alpha = ex2_approx(m - m_tile);
+          m = m_tile;
+          need = true;
+        }
+        float sum = 0.f;
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int i = 0; i < BN / 2; ++i) {
+          const float p0 = ex2_approx(fmaf(sv[2 * i], scale_log2, -m));
+          const float p1 = ex2_approx(fmaf(sv[2 * i + 1], scale_log2, -m));
+          sum += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        l = l * alpha + sum;
+        // P (bf16 pairs) into the first 64 columns of this tile's S region.
+        tmem_st32(lane_base + colS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(lane_base + colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        if (__any_sync(0xffffffffu, need)) {
+          // O_t holds sum_{j'<j} P V, and PV_t(j-1) has completed: it precedes S_t(j).
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + colO + c * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(lane_base + colO + c * 32, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[t]);
+      }
+      if (!ok) break;
+      // -------------------------------------------------------------- epilogue
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[t], units & 1, ab, status, timeout_ns));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t s_addr = lane_base + (j & 1) * BN;
-      float sv[BN];
+      uint32_t o[D];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld32(s_addr + c * 32, u);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(u[i]);
-      }
-      const int k0 = j * BN;
-      const bool diag = CAUSAL && (k0 + BN - 1 > q0);
-      const bool tail = (k0 + BN > N);
-      if (diag || tail) {
-        const int lim = min(CAUSAL ? row : N - 1, N - 1) - k0;  // last visible column
-#pragma unroll
-        for (int i = 0; i < BN; ++i)
-          if (i > lim) sv[i] = -INFINITY;
-      }
-      float mx = sv[0];
-#pragma unroll
-      for (int i = 1; i < BN; ++i) mx = fmaxf(mx, sv[i]);
-      const float m_tile = mx * scale_log2;
-      float alpha = 1.f;
-      bool need = false;
-      if (m == -INFINITY) {
-        m = m_tile;
-      } else if (m_tile - m > kRescaleThreshold) {
-        alpha = ex2_approx(m - m_tile);
-        m = m_tile;
-        need = true;
-      }
-      float sum = 0.f;
-      uint32_t pk[BN / 2];
-#pragma unroll
-      for (int i = 0; i < BN / 2; ++i) {
-        const float p0 = ex2_approx(fmaf(sv[2 * i], scale_log2, -m));
-        const float p1 = ex2_approx(fmaf(sv[2 * i + 1], scale_log2, -m));
-        sum += p0 + p1;
-        pk[i] = pack_bf16x2(p0, p1);
-      }
-      l = l * alpha + sum;
-      {
-        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
-        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
-        tmem_st32(s_addr, lo);
-        tmem_st32(s_addr + 32, hi);
-      }
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // O holds sum_{j'<j} P V; make sure the last PV landed before rescaling it.
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(&bars->o_done, (j - 1) & 1, ab, status, timeout_ns));
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t u[32];
-          tmem_ld32(lane_base + kColO + c * 32, u);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-          tmem_st32(lane_base + kColO + c * 32, u);
-        }
-      }
-      tmem_st_wait();
+      for (int c = 0; c < D / 64; ++c)
+        tmem_ld64(lane_base + colO + 64 * c, *reinterpret_cast<uint32_t(*)[64]>(&o[64 * c]));
       tc_fence_before();
-      mbar_arrive(&bars->p_full[j & 1]);
+      mbar_arrive(&bars->o_free[t]);  // the next unit's first PV may overwrite O_t now
+      ++units;
+      if (row < N) {
+        const float inv_l = 1.f / l;
+        __nv_bfloat16* orow = out + ((static_cast<size_t>(b) * N + row) * H + h) * D;
+#pragma unroll
+        for (int c8 = 0; c8 < D / 8; ++c8)
+          reinterpret_cast<uint4*>(orow)[c8] = make_uint4(
+              pack_bf16x2(__uint_as_float(o[8 * c8 + 0]) * inv_l, __uint_as_float(o[8 * c8 + 1]) * inv_l),
+              pack_bf16x2(__uint_as_float(o[8 * c8 + 2]) * inv_l, __uint_as_float(o[8 * c8 + 3]) * inv_l),
+              pack_bf16x2(__uint_as_float(o[8 * c8 + 4]) * inv_l, __uint_as_float(o[8 * c8 + 5]) * inv_l),
+              pack_bf16x2(__uint_as_float(o[8 * c8 + 6]) * inv_l, __uint_as_float(o[8 * c8 + 7]) * inv_l));
+        lse[static_cast<size_t>(x.bh) * N + row] = (m + __log2f(l)) * 0.69314718055994531f;
+      }
     }
-    // ---------------------------------------------------------------- epilogue
-    if (ok) ok = __all_sync(0xffffffffu,
-                            mbar_wait(&bars->o_done, (nkv - 1) & 1, ab, status, timeout_ns));
-    if (ok) {
-      tc_fence_after();
-      const float inv_l = 1.f / l;
-      __nv_bfloat16* orow = out + ((static_cast<size_t>(b) * N + row) * H + h) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld32(lane_base + kColO + c * 32, u);
-        uint32_t pkd[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pkd[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
-        if (row < N) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            dst[v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+  } else {
+    regs_set<kRegsLaunch, kRegsOther>();
+    if (warp == kWarpLoad) {
+      // ---------------------------------------------------------------- TMA producer
+      if (lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        const uint64_t pol_q = policy_evict_first();
+        const uint64_t pol_kv = policy_evict_last();
+        int g = 0;      // K/V tiles issued so far (ring position)
+        int units = 0;  // units started
+        bool ok = true;
+        for (int r = 0; ok; ++r) {
+          const int u = unit_of_round(r, G);
+          if (u >= num_units) break;
+          const Unit x = decode_unit<CAUSAL>(u, BH, num_pairs);
+          const int b = x.bh / H, h = x.bh % H;
+          if (units > 0 &&
+              !(ok = mbar_wait(&bars->q_empty, (units - 1) & 1, ab, status, timeout_ns)))
+            break;
+          mbar_arrive_expect_tx(&bars->q_full, 2 * C::kTileBytes);
+          for (int t = 0; t < 2; ++t)
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &tm_q, &bars->q_full,
+                          c * 64, h, (2 * x.pair + t) * BM, b, pol_q);
+          ++units;
+          const int nkv = kv_tiles<CAUSAL>(x.pair, 1, kv_total);
+          for (int j = 0; j < nkv; ++j, ++g) {
+            const int s = g % C::kStages;
+            const uint32_t ph = ((g / C::kStages) - 1) & 1;
+            if (g >= C::kStages &&
+                !(ok = mbar_wait(&bars->k_empty[s], ph, ab, status, timeout_ns)))
+              break;
+            mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes);
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_4d(sK + s * C::kTileBytes + c * C::kChunkBytes, &tm_k, &bars->k_full[s],
+                          c * 64, h, j * BN, b, pol_kv);
+            if (g >= C::kStages &&
+                !(ok = mbar_wait(&bars->v_empty[s], ph, ab, status, timeout_ns))) {
+              ++g;  // K of this tile is in flight: count it for the drain below
+              break;
+            }
+            mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_4d(sV + s * C::kTileBytes + c * C::kChunkBytes, &tm_v, &bars->v_full[s],
+                          c * 64, h, j * BN, b, pol_kv);
+          }
+        }
+        // Drain: no copy into shared memory may still be in flight when the CTA exits.
+        // Only the last Q pair and the last kStages K/V tiles can be outstanding.  (On the
+        // abort path a V copy may not have been issued; its wait then runs out harmlessly.)
+        Abort local{0};
+        if (units > 0) mbar_wait(&bars->q_full, (units - 1) & 1, &local, status, timeout_ns);
+        for (int gg = max(0, g - C::kStages); gg < g; ++gg) {
+          mbar_wait(&bars->k_full[gg % C::kStages], (gg / C::kStages) & 1, &local, status,
+                    timeout_ns);
+          if (ok || gg < g - 1)
+            mbar_wait(&bars->v_full[gg % C::kStages], (gg / C::kStages) & 1, &local, status,
+                      timeout_ns);
         }
       }
-      if (row < N)
-        lse[(static_cast<size_t>(b) * H + h) * N + row] = (m + __log2f(l)) * 0.69314718055994531f;
+    } else if (warp == kWarpMma) {
+      // ---------------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
+        constexpr uint32_t idesc_o = idesc_bf16_f32(BM, D, 0, 1);
+        const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+        int g = 0;            // K/V tiles consumed so far (ring position)
+        int units = 0;        // units finished
+        int np[2] = {0, 0};   // p_full phases consumed per tile
+        bool ok = true;
+        auto issue_s = [&](int t, int s) {  // S_t = Q_t K^T (both K-major over the head dim)
+          const uint32_t kb = aK + s * C::kTileBytes;
+          const uint32_t qb = aQ + t * C::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+            umma_ss(tbase + BN * t, sdesc_sw128(qb + off, 16, 1024),
+                    sdesc_sw128(kb + off, 16, 1024), idesc_s, kk > 0);
+          }
+          umma_commit(&bars->s_full[t]);
+        };
+        auto issue_pv = [&](int t, int s, bool first) {  // O_t += P_t V (P from TMEM)
+          const uint32_t vb = aV + s * C::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            umma_ts(tbase + C::kColO + D * t, tbase + BN * t + kk * 8,
+                    sdesc_sw128(vb + kk * 2048, C::kChunkBytes, 1024), idesc_o,
+                    (!first || kk > 0) ? 1u : 0u);
+        };
+        for (int r = 0; ok; ++r) {
+          const int u = unit_of_round(r, G);
+          if (u >= num_units) break;
+          const Unit x = decode_unit<CAUSAL>(u, BH, num_pairs);
+          const int nkv0 = kv_tiles<CAUSAL>(x.pair, 0, kv_total);
+          const int nkv1 = kv_tiles<CAUSAL>(x.pair, 1, kv_total);
+          if (!(ok = mbar_wait(&bars->q_full, units & 1, ab, status, timeout_ns))) break;
+          {  // prologue: S0(0), S1(0)
+            const int s = g % C::kStages;
+            if (!(ok = mbar_wait(&bars->k_full[s], (g / C::kStages) & 1, ab, status, timeout_ns)))
+              break;
+            tc_fence_after();
+            issue_s(0, s);
+            issue_s(1, s);
+            umma_commit(&bars->k_empty[s]);
+            if (nkv1 == 1) umma_commit(&bars->q_empty);  // last S products of this unit
+          }
+          for (int j = 0; ok && j < nkv1; ++j) {
+            const int s = (g + j) % C::kStages;
+            const int s1 = (g + j + 1) % C::kStages;
+            const bool more = j + 1 < nkv1;
+            if (!(ok = mbar_wait(&bars->v_full[s], ((g + j) / C::kStages) & 1, ab, status,
+                                 timeout_ns)))
+              break;
+            if (more && !(ok = mbar_wait(&bars->k_full[s1], ((g + j + 1) / C::kStages) & 1, ab,
+                                         status, timeout_ns)))
+              break;
+            if (j < nkv0) {  // tile 0: PV0(j), S0(j+1)
+              if (j == 0 && units > 0 &&
+                  !(ok = mbar_wait(&bars->o_free[0], (units - 1) & 1, ab, status, timeout_ns)))
+                break;
+              if (!(ok = mbar_wait(&bars->p_full[0], np[0] & 1, ab, status, timeout_ns))) break;
+              ++np[0];
+              tc_fence_after();
+              issue_pv(0, s, j == 0);
+              if (j + 1 < nkv0) {
+                issue_s(0, s1);
+              } else {
+                umma_commit(&bars->o_done[0]);
+              }
+            }
+            // tile 1: PV1(j), S1(j+1)
+            if (j == 0 && units > 0 &&
+                !(ok = mbar_wait(&bars->o_free[1], (units - 1) & 1, ab, status, timeout_ns)))
+              break;
+            if (!(ok = mbar_wait(&bars->p_full[1], np[1] & 1, ab, status, timeout_ns))) break;
+            ++np[1];
+            tc_fence_after();
+            issue_pv(1, s, j == 0);
+            umma_commit(&bars->v_empty[s]);
+            if (more) {
+              issue_s(1, s1);
+              umma_commit(&bars->k_empty[s1]);
+              if (j + 2 == nkv1) umma_commit(&bars->q_empty);  // last S products of this unit
+            } else {
+              umma_commit(&bars->o_done[1]);
+            }
+          }
+          g += nkv1;
+          ++units;
+        }
+        // Drain every MMA this thread issued before TMEM is released.
+        umma_commit(&bars->drain);
+        Abort local{0};
+        mbar_wait(&bars->drain, 0, &local, status, timeout_ns);
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     __syncwarp();
     tmem_dealloc(tbase, kTmemCols);
   }
@@ -322,16 +445,23 @@ template <int D, bool CAUSAL>
 static cudaError_t launch_t(const FwdArgs& a, cudaStream_t st) {
   using C = Cfg<D>;
   auto kern = fwd_kernel<D, CAUSAL>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
+  // The setmaxnreg split assumes the kernel launches with exactly kRegsLaunch registers per
+  // thread; with fewer, the softmax warpgroups' increase could never be satisfied.
+  cudaFuncAttributes fa_attr;
+  cudaError_t e = cudaFuncGetAttributes(&fa_attr, kern);
   if (e != cudaSuccess) return e;
-  const int num_qtiles = (a.N + BM - 1) / BM;
-  const long long grid = static_cast<long long>(a.B) * a.H * num_qtiles;
-  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  if (fa_attr.numRegs != static_cast<int>(kRegsLaunch)) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int num_pairs = (a.N + 2 * BM - 1) / (2 * BM);
+  const long long units = static_cast<long long>(a.B) * a.H * num_pairs;
+  if (units > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const int grid = static_cast<int>(std::min<long long>(units, a.num_sms));
   const float scale_log2 = a.scale * 1.4426950408889634f;
-  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, st>>>(
-      a.tm_q, a.tm_k, a.tm_v, static_cast<__nv_bfloat16*>(a.o), a.lse, a.B, a.H, a.N, scale_log2,
-      num_qtiles, a.status, kDefaultWaitTimeoutNs);
+  kern<<<grid, kThreads, C::kSmemBytes, st>>>(a.tm_q, a.tm_k, a.tm_v,
+                                              static_cast<__nv_bfloat16*>(a.o), a.lse, a.B, a.H,
+                                              a.N, scale_log2, num_pairs, a.status,
+                                              kDefaultWaitTimeoutNs);
   return cudaGetLastError();
 }
 
