@@ -103,7 +103,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -395,17 +395,91 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep(path: str, reps: int = 20, warmup: int = 3):
+    """Times every workload of the benchmark sweep (forward-only configs: fa_fwd; forward +
+    backward configs: fa_fwd and fa_bwd separately) and writes one JSON line per workload
+    to `path`.  Median of `reps` CUDA-event timed launches after `warmup`."""
+    import torch
+    from exact_io_aware_88_b200 import fa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = measured_peaks()
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts), min(ts)
+
+    with open(path, "w") as out:
+        for w in synthetic.all_workloads():
+            t = synthetic.draw_workload(w, with_grad=w.backward)
+            B, N, H, d = w.B, w.N, w.H, w.d
+            q, k, v = (t[n].to(dev) for n in ("q", "k", "v"))
+            o = torch.empty_like(q)
+            lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+            f = fa.fa_fwd_f32 if w.dtype == "f32" else fa.fa_fwd
+            fwd = lambda: f(q, k, v, o, lse, B, H, N, d, w.causal, w.scale, stream)
+            assert fwd() == 0
+            med, best = timed(fwd)
+            elem = 4 if w.dtype == "f32" else 2
+            hbm_floor = (4 * B * N * H * d * elem + 4 * B * H * N) / (hbm * 1e9) * 1e3  # ms
+            rec = {"workload": w.label(), "pass": "fwd", "ms": round(med, 4), "ms_best": round(best, 4),
+                   "tflops": round(w.fwd_flops() / (med * 1e-3) / 1e12, 1),
+                   "frac_of_burst_peak": round(w.fwd_flops() / (med * 1e-3) / 1e12 / burst, 4),
+                   "hbm_floor_ms": round(hbm_floor, 4), "peak_source": peak_src}
+            out.write(json.dumps(rec) + "\n")
+            print(json.dumps(rec), file=sys.stderr)
+            if w.backward:
+                dO = t["dO"].to(dev)
+                dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+                nb = fa.fa_bwd_workspace_bytes(B, H, N, d)
+                ws = torch.empty(nb, device=dev, dtype=torch.uint8)
+                bwd = lambda: fa.fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, w.causal,
+                                        w.scale, ws, nb, stream)
+                assert bwd() == 0
+                med, best = timed(bwd)
+                rec = {"workload": w.label(), "pass": "bwd", "ms": round(med, 4),
+                       "ms_best": round(best, 4),
+                       "tflops": round(w.bwd_flops() / (med * 1e-3) / 1e12, 1),
+                       "frac_of_burst_peak": round(w.bwd_flops() / (med * 1e-3) / 1e12 / burst, 4),
+                       "peak_source": peak_src}
+                out.write(json.dumps(rec) + "\n")
+                print(json.dumps(rec), file=sys.stderr)
+                del dO, dq, dk, dv, ws
+            del q, k, v, o, lse, t
+            torch.cuda.empty_cache()
+    if fa.fa_read_device_status(stream) != 0:
+        raise RuntimeError("device status word reports a timeout")
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=250)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--N", type=int, default=16384, choices=[1024, 2048, 4096, 8192, 16384, 65536])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", metavar="PATH", default=None,
+                    help="time every workload of the benchmark sweep into PATH (JSON lines) "
+                         "instead of the single-step measurement")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.sweep:
+        run_sweep(args.sweep)
+        return
     rank, world, local_rank = dist_env()
     if world != args.gpus and world > 1:
         print(f"warning: WORLD_SIZE={world} but --gpus={args.gpus}", file=sys.stderr)

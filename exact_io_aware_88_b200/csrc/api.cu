@@ -355,6 +355,15 @@ int fa_debug_umma_tile(const void* a, const void* b, float* c, int n, int k, int
       fa::launch_debug_umma(a, b, c, n, k, mode, di.status, static_cast<cudaStream_t>(stream)));
 }
 
+int fa_debug_exp2(const float* x, float* y_poly, float* y_hw, int n, void* stream) {
+  if (!x || !y_poly || !y_hw || n < 1 || n > (1 << 28)) return FA_ERR_INVALID_ARG;
+  if (!aligned(x, 4) || !aligned(y_poly, 4) || !aligned(y_hw, 4)) return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  return from_cuda(fa::launch_debug_exp2(x, y_poly, y_hw, n, static_cast<cudaStream_t>(stream)));
+}
+
 int fa_debug_wait_timeout(long long timeout_ns, void* stream) {
   if (timeout_ns < 1000 || timeout_ns > 10000000000LL) return FA_ERR_INVALID_ARG;
   DeviceInfo di;

@@ -133,7 +133,29 @@ __global__ void wait_timeout_kernel(uint64_t timeout_ns, int* status) {
   mbar_wait(&bar, 0, &ab, status, timeout_ns);
 }
 
+// y_poly[i] = software exp2 (exp2_poly2), y_hw[i] = hardware ex2.approx, of x[i].
+__global__ void exp2_kernel(const float* __restrict__ x, float* __restrict__ y_poly,
+                            float* __restrict__ y_hw, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.f;
+  float p0, p1;
+  f2_unpack(exp2_poly2(f2_pack(a, b)), p0, p1);
+  y_poly[i] = p0;
+  y_hw[i] = ex2_approx(a);
+  if (i + 1 < n) {
+    y_poly[i + 1] = p1;
+    y_hw[i + 1] = ex2_approx(b);
+  }
+}
+
 }  // namespace dbg
+
+cudaError_t launch_debug_exp2(const float* x, float* y_poly, float* y_hw, int n, cudaStream_t s) {
+  const int pairs = (n + 1) / 2;
+  dbg::exp2_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(x, y_poly, y_hw, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_debug_umma(const void* a, const void* b, float* c, int n, int k, int mode,
                               int* status, cudaStream_t s) {

@@ -339,6 +339,73 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// ----------------------------------------------------------------------------- f32x2 math
+// sm_100 executes some fp32 operations on pairs packed in a 64-bit register (one issue slot
+// for two results).  Pairs are held as uint64_t: low half = first element.
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Software exp2 of a pair, on the FMA pipe instead of the MUFU unit.
+// Method (Cody-Waite range reduction + minimax polynomial): x = n + f with n = round(x)
+// (found by adding 1.5*2^23, whose low mantissa bits then hold n) and f in [-1/2, 1/2];
+// 2^f ~ p(f), the degree-3 polynomial minimising the maximum relative error on [-1/2, 1/2]
+// (Remez exchange, coefficients from gen_exp2_poly.py: max relative error 7.5e-5); then n
+// is added to the exponent field of p(f).  Inputs are clamped to >= -125 so the exponent
+// stays in the normal range; below that the result is ~2^-125 instead of 0, so callers use
+// the hardware exp2 where exact zeros (masked logits) are required.
+constexpr float kExp2C0 = 0.999928057f;
+constexpr float kExp2C1 = 0.693260968f;
+constexpr float kExp2C2 = 0.242611125f;
+constexpr float kExp2C3 = 0.0551716685f;
+constexpr float kExp2Magic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+  float a, b;
+  f2_unpack(x, a, b);
+  x = f2_pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
+  const uint64_t magic = f2_pack(kExp2Magic, kExp2Magic);
+  const uint64_t t = f2_add(x, magic);          // low bits: n = round(x)
+  const uint64_t f = f2_sub(x, f2_sub(t, magic));  // x - n, in [-1/2, 1/2]
+  uint64_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+  uint32_t t0, t1, p0, p1;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(t0), "=r"(t1) : "l"(t));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(p));
+  p0 += t0 << 23;  // (bits of 1.5*2^23 + n) << 23 == n << 23 (mod 2^32)
+  p1 += t1 << 23;
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(p0), "r"(p1));
+  return r;
+}
+
 // Byte offset of 16-byte chunk `chunk` of row `row` inside a 128-byte-swizzled tile
 // whose rows are 128 bytes long (1024-byte aligned base).
 __host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {

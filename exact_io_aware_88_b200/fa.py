@@ -73,13 +73,16 @@ _lib.fa_version.argtypes = []
 _lib.fa_version.restype = _I
 _lib.fa_debug_umma_tile.argtypes = [_P, _P, _P, _I, _I, _I, _P]
 _lib.fa_debug_umma_tile.restype = _I
+_lib.fa_debug_exp2.argtypes = [_P, _P, _P, _I, _P]
+_lib.fa_debug_exp2.restype = _I
 _lib.fa_debug_wait_timeout.argtypes = [ctypes.c_longlong, _P]
 _lib.fa_debug_wait_timeout.restype = _I
 
 # Every symbol the C headers declare, for the ABI self-check.
 EXPORTED = sorted(["fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_kv",
                    "fa_bwd_dq_convert", "fa_bwd_noalloc", "fa_fwd_f32", "fa_read_device_status", "fa_status_string",
-                   "fa_version", "fa_debug_umma_tile", "fa_debug_wait_timeout"])
+                   "fa_version", "fa_debug_umma_tile", "fa_debug_wait_timeout",
+                   "fa_debug_exp2"])
 
 
 def _ptr(x) -> Optional[int]:
@@ -164,6 +167,10 @@ def fa_read_device_status(stream=None) -> int:
 
 def fa_debug_umma_tile(a, b, c, n, k, mode, stream=None) -> int:
     return _lib.fa_debug_umma_tile(_ptr(a), _ptr(b), _ptr(c), n, k, mode, _stream(stream))
+
+
+def fa_debug_exp2(x, y_poly, y_hw, n, stream=None) -> int:
+    return _lib.fa_debug_exp2(_ptr(x), _ptr(y_poly), _ptr(y_hw), int(n), _stream(stream))
 
 
 def fa_debug_wait_timeout(timeout_ns, stream=None) -> int:

@@ -23,6 +23,11 @@ extern "C" {
 int fa_debug_umma_tile(const void* a, const void* b, float* c, int n, int k, int mode,
                        void* stream);
 
+/* Evaluates, for each of the n fp32 inputs x[i] (device pointers), the kernels' software
+ * exp2 (range reduction to [-1/2, 1/2] + degree-3 minimax polynomial on the FMA pipe) into
+ * y_poly[i] and the hardware ex2.approx into y_hw[i].  1 <= n <= 2^28. */
+int fa_debug_exp2(const float* x, float* y_poly, float* y_hw, int n, void* stream);
+
 /* Launches one CTA whose only work is a bounded wait on an mbarrier that nothing ever
  * arrives at.  The wait gives up after `timeout_ns` nanoseconds (1e3 .. 1e10), records
  * FA_ERR_TIMEOUT in the device status word and the CTA exits normally.  Read the result

@@ -40,6 +40,26 @@ def test_umma_tile(fa, mode, n, k):
     np.testing.assert_allclose(C.double().cpu().numpy(), ref.numpy(), atol=2e-3, rtol=1e-5)
 
 
+def test_software_exp2_within_its_error_bound(fa):
+    # Range the kernels feed it: logits minus a running max, i.e. <= 8 (stale max) and down
+    # to the clamp at -125; plus the exact integers where the reduction is trivial.
+    x = np.concatenate([np.linspace(-125.0, 8.0, 1_000_003), np.arange(-125, 9, dtype=np.float64),
+                        np.random.default_rng(0).uniform(-30, 8, 100_000)]).astype(np.float32)
+    dx = torch.from_numpy(x).cuda()
+    yp, yh = torch.empty_like(dx), torch.empty_like(dx)
+    assert fa.fa_debug_exp2(dx, yp, yh, x.size) == 0
+    torch.cuda.synchronize()
+    exact = np.exp2(x.astype(np.float64))
+    rel_poly = np.abs(yp.cpu().numpy().astype(np.float64) / exact - 1.0)
+    rel_hw = np.abs(yh.cpu().numpy().astype(np.float64) / exact - 1.0)
+    # minimax bound of the polynomial (7.5e-5) plus fp32 rounding of the reduction
+    assert rel_poly.max() < 1e-4, rel_poly.max()
+    # the hardware exp2 is the reference scale for what the kernels accept elsewhere
+    assert rel_hw.max() < 1e-5
+    # bf16 (the precision P is stored in) cannot tell them apart most of the time
+    assert np.mean(rel_poly < 2.0 ** -9) == 1.0
+
+
 def test_bounded_wait_times_out_and_reports(fa):
     assert fa.fa_debug_wait_timeout(50_000_000) == 0
     assert fa.fa_read_device_status() == fa.FA_ERR_TIMEOUT
