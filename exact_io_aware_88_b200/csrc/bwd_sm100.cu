@@ -217,10 +217,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float4 l4 = gL[c / 4];
           const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float e = ex2_approx(fmaf(__uint_as_float(su[c + u]), scale_log2, -lv[u]));
-            p[c + u] = (row_dead || c + u < first_vis || c + u > last_vis) ? 0.f : e;
-          }
+          for (int u = 0; u < 4; ++u)
+            p[c + u] = ex2_approx(fmaf(__uint_as_float(su[c + u]), scale_log2, -lv[u]));
+        }
+        // Masks only where the tile needs them (diagonal or tail tiles; decided per warp so
+        // the common, unmasked tiles pay nothing).
+        const bool need_mask = row_dead || first_vis > 0 || last_vis < 63;
+        if (__any_sync(0xffffffffu, need_mask)) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (row_dead || c < first_vis || c > last_vis) p[c] = 0.f;
         }
       }
       {
@@ -394,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Per query tile n (rows i = i_begin + n), in issue order:
       //   [p_ready n]  dV += P^T_n dO_n                 -> releases dO_n
       //                S^T_{n+1} = K Q_{n+1}^T (R1)      (P^T_n already consumed, in order)
-      //   [ds_ready n] dK += dS^T_n Q_n ; dQ_n = dS_n K (R2) -> releases Q_n
+      //   [ds_ready n] dQ_n = dS_n K (R2) ; dK += dS^T_n Q_n -> releases Q_n
       //   [dq_empty n] dP^T_{n+1} = V dO_{n+1}^T (R2)
       // so the next S^T and dV overlap the dS computation, and the dQ drain only gates dP.
       if (lane == 0) {
@@ -452,13 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (n + 1 < nq && !issue_s(n + 1)) break;
           if (!mbar_wait(&bars->ds_ready, n & 1, ab, status, timeout_ns)) break;
           tc_fence_after();
-          // dK_j += dS^T Q_i   (A = dS^T K-major over the query index, B = Q_i MN-major)
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint32_t aoff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-            umma_ss(tbase + C::kColDK, sdesc_sw128(aDS + aoff, 16, 1024),
-                    sdesc_sw128(qb + kk * 2048, C::kChunkBytes, 1024), id_dkdv, (n > 0 || kk > 0));
-          }
+          // dQ first: only its drain gates the next dP^T, so dK runs on the tensor pipe
+          // while the drain warps empty the dQ columns.
           if constexpr (kDqTransposed<D>) {
             // dQ_i^T = K_j^T dS^T   (A = K_j read MN-major over the head dim, B = dS^T
             // MN-major over the query index): TMEM lane = head-dim index, column = query.
@@ -474,6 +475,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                       sdesc_sw128(aK + kk * 2048, C::kChunkBytes, 1024), id_dq, kk > 0);
           }
           umma_commit(&bars->dq_full);
+          // dK_j += dS^T Q_i   (A = dS^T K-major over the query index, B = Q_i MN-major)
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint32_t aoff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+            umma_ss(tbase + C::kColDK, sdesc_sw128(aDS + aoff, 16, 1024),
+                    sdesc_sw128(qb + kk * 2048, C::kChunkBytes, 1024), id_dkdv, (n > 0 || kk > 0));
+          }
           umma_commit(&bars->q_empty[sq]);
           if (n + 1 < nq && !issue_dp(n + 1)) break;
         }
