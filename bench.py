@@ -456,6 +456,18 @@ def run_sweep(path: str, reps: int = 20, warmup: int = 3):
                        "peak_source": peak_src}
                 out.write(json.dumps(rec) + "\n")
                 print(json.dumps(rec), file=sys.stderr)
+                det = lambda: fa.fa_bwd_deterministic(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d,
+                                                      w.causal, w.scale, ws, nb, stream)
+                assert det() == 0
+                med, best = timed(det)
+                rec = {"workload": w.label(), "pass": "bwd_deterministic", "ms": round(med, 4),
+                       "ms_best": round(best, 4),
+                       "tflops": round(w.bwd_flops() / (med * 1e-3) / 1e12, 1),
+                       "frac_of_burst_peak": round(w.bwd_flops() / (med * 1e-3) / 1e12 / burst, 4),
+                       "peak_source": peak_src,
+                       "note": "FLOPs counted as 2.5x forward; the kernels do 3.5x (dQ recomputes S, dP)"}
+                out.write(json.dumps(rec) + "\n")
+                print(json.dumps(rec), file=sys.stderr)
                 del dO, dq, dk, dv, ws
             del q, k, v, o, lse, t
             torch.cuda.empty_cache()

@@ -228,8 +228,22 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = from_cuda(fa::launch_bwd_pre(a, st)))) return rc;
-  if ((rc = from_cuda(fa::launch_bwd_main(a, st)))) return rc;
+  if ((rc = from_cuda(fa::launch_bwd_main(a, st, true)))) return rc;
   return from_cuda(fa::launch_bwd_convert(a, st));
+}
+
+int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
+                         int H, int N, int d, int causal, float scale, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  fa::BwdArgs a;
+  int rc = bwd_prepare(kStagePre | kStageMain | kStageConvert, q, k, v, o, lse, dO, dq, dk, dv, B,
+                       H, N, d, causal, scale, workspace, workspace_bytes, &a);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = from_cuda(fa::launch_bwd_pre(a, st)))) return rc;
+  if ((rc = from_cuda(fa::launch_bwd_main(a, st, false)))) return rc;
+  return from_cuda(fa::launch_bwd_dq(a, st));
 }
 
 int fa_bwd_preprocess(const void* o, const float* lse, const void* dO, int B, int H, int N, int d,
@@ -248,7 +262,7 @@ int fa_bwd_kv(const void* q, const void* k, const void* v, const void* dO, void*
   int rc = bwd_prepare(kStageMain, q, k, v, nullptr, nullptr, dO, nullptr, dk, dv, B, H, N, d,
                        causal, scale, workspace, workspace_bytes, &a);
   if (rc) return rc;
-  return from_cuda(fa::launch_bwd_main(a, static_cast<cudaStream_t>(stream)));
+  return from_cuda(fa::launch_bwd_main(a, static_cast<cudaStream_t>(stream), true));
 }
 
 int fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, void* workspace,
@@ -307,7 +321,7 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = from_cuda(fa::launch_bwd_pre(a, st)))) return rc;
-  if ((rc = from_cuda(fa::launch_bwd_main(a, st)))) return rc;
+  if ((rc = from_cuda(fa::launch_bwd_main(a, st, true)))) return rc;
   return from_cuda(fa::launch_bwd_convert(a, st));
 }
 

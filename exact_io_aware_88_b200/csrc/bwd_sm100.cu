@@ -109,7 +109,9 @@ constexpr bool kDqTransposed = (D == 128);
 // S^T region, i.e. inside the S^T columns it has already read.
 __device__ __forceinline__ uint32_t p_col(int kk) { return 64u * (kk >> 2) + 8u * (kk & 3); }
 
-template <int D, bool CAUSAL>
+// WITH_DQ = false drops the dQ product and its drain (dQ then comes from the separate,
+// deterministic per-query-tile kernel in bwd_dq_sm100.cu).
+template <int D, bool CAUSAL, bool WITH_DQ>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -301,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;  // query row within the tile
     const uint32_t lane_base = tbase + (static_cast<uint32_t>(quarter * 32) << 16);
-    for (int n = 0; n < nq; ++n) {
+    for (int n = 0; WITH_DQ && n < nq; ++n) {
       const int q = (i_begin + n) * BN + r;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_full, n & 1, ab, status, timeout_ns));
       if (!ok) break;
@@ -430,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int sd = n % C::kDOStages;
           if (!mbar_wait(&bars->do_full[sd], (n / C::kDOStages) & 1, ab, status, timeout_ns))
             return false;
-          if (n > 0 && !mbar_wait(&bars->dq_empty, (n - 1) & 1, ab, status, timeout_ns))
+          if (WITH_DQ && n > 0 && !mbar_wait(&bars->dq_empty, (n - 1) & 1, ab, status, timeout_ns))
             return false;
           tc_fence_after();
           const uint32_t dob = aDO + sd * C::kTileBytes;
@@ -460,7 +462,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           // dQ first: only its drain gates the next dP^T, so dK runs on the tensor pipe
           // while the drain warps empty the dQ columns.
-          if constexpr (kDqTransposed<D>) {
+          if constexpr (!WITH_DQ) {
+          } else if constexpr (kDqTransposed<D>) {
             // dQ_i^T = K_j^T dS^T   (A = K_j read MN-major over the head dim, B = dS^T
             // MN-major over the query index): TMEM lane = head-dim index, column = query.
 #pragma unroll
@@ -474,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               umma_ss(tbase + C::kColDP, sdesc_sw128(aDS + kk * 2048, C::kChunkBytes, 1024),
                       sdesc_sw128(aK + kk * 2048, C::kChunkBytes, 1024), id_dq, kk > 0);
           }
-          umma_commit(&bars->dq_full);
+          if constexpr (WITH_DQ) umma_commit(&bars->dq_full);
           // dK_j += dS^T Q_i   (A = dS^T K-major over the query index, B = Q_i MN-major)
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
@@ -599,11 +602,11 @@ static cudaError_t launch_pre_t(const BwdArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool WITH_DQ>
 static cudaError_t launch_main_t(const BwdArgs& a, cudaStream_t st) {
   using C = Cfg<D>;
   const int n_pad = (a.N + 127) / 128 * 128;
-  auto kern = bwd_main_kernel<D, CAUSAL>;
+  auto kern = bwd_main_kernel<D, CAUSAL, WITH_DQ>;
   // The setmaxnreg split assumes the kernel launches with exactly kRegsLaunch registers per
   // thread; with fewer, the increasing warpgroups could never be satisfied.
   cudaFuncAttributes fa_attr;
@@ -638,10 +641,19 @@ cudaError_t launch_bwd_pre(const BwdArgs& a, cudaStream_t s) {
   return a.d == 64 ? bwd::launch_pre_t<64>(a, s) : bwd::launch_pre_t<128>(a, s);
 }
 
-cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t s) {
+cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t s, bool with_dq) {
+  if (with_dq) {
+    if (a.d == 64)
+      return a.causal ? bwd::launch_main_t<64, true, true>(a, s)
+                      : bwd::launch_main_t<64, false, true>(a, s);
+    return a.causal ? bwd::launch_main_t<128, true, true>(a, s)
+                    : bwd::launch_main_t<128, false, true>(a, s);
+  }
   if (a.d == 64)
-    return a.causal ? bwd::launch_main_t<64, true>(a, s) : bwd::launch_main_t<64, false>(a, s);
-  return a.causal ? bwd::launch_main_t<128, true>(a, s) : bwd::launch_main_t<128, false>(a, s);
+    return a.causal ? bwd::launch_main_t<64, true, false>(a, s)
+                    : bwd::launch_main_t<64, false, false>(a, s);
+  return a.causal ? bwd::launch_main_t<128, true, false>(a, s)
+                  : bwd::launch_main_t<128, false, false>(a, s);
 }
 
 cudaError_t launch_bwd_convert(const BwdArgs& a, cudaStream_t s) {

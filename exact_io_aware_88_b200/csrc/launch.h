@@ -39,7 +39,8 @@ struct BwdArgs {
 
 cudaError_t launch_fwd_sm100(const FwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_pre(const BwdArgs& a, cudaStream_t s);
-cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t s, bool with_dq);
+cudaError_t launch_bwd_dq(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_convert(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
                            int B, int H, int N, int d, int causal, float scale, cudaStream_t s);

@@ -55,6 +55,8 @@ _lib.fa_bwd_workspace_bytes.argtypes = [_I, _I, _I, _I]
 _lib.fa_bwd_workspace_bytes.restype = _SZ
 _lib.fa_bwd.argtypes = [_P] * 9 + [_I, _I, _I, _I, _I, _F, _P, _SZ, _P]
 _lib.fa_bwd.restype = _I
+_lib.fa_bwd_deterministic.argtypes = [_P] * 9 + [_I, _I, _I, _I, _I, _F, _P, _SZ, _P]
+_lib.fa_bwd_deterministic.restype = _I
 _lib.fa_bwd_preprocess.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]
 _lib.fa_bwd_preprocess.restype = _I
 _lib.fa_bwd_kv.argtypes = [_P] * 6 + [_I, _I, _I, _I, _I, _F, _P, _SZ, _P]
@@ -79,7 +81,7 @@ _lib.fa_debug_wait_timeout.argtypes = [ctypes.c_longlong, _P]
 _lib.fa_debug_wait_timeout.restype = _I
 
 # Every symbol the C headers declare, for the ABI self-check.
-EXPORTED = sorted(["fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_kv",
+EXPORTED = sorted(["fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess", "fa_bwd_kv",
                    "fa_bwd_dq_convert", "fa_bwd_noalloc", "fa_fwd_f32", "fa_read_device_status", "fa_status_string",
                    "fa_version", "fa_debug_umma_tile", "fa_debug_wait_timeout",
                    "fa_debug_exp2"])
@@ -123,6 +125,14 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, workspace
     return _lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
                        _ptr(dk), _ptr(dv), B, H, N, d, int(causal), float(scale),
                        _ptr(workspace), int(workspace_bytes), _stream(stream))
+
+
+def fa_bwd_deterministic(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, workspace,
+                         workspace_bytes, stream=None) -> int:
+    return _lib.fa_bwd_deterministic(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO),
+                                     _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, int(causal),
+                                     float(scale), _ptr(workspace), int(workspace_bytes),
+                                     _stream(stream))
 
 
 def fa_bwd_preprocess(o, lse, dO, B, H, N, d, workspace, workspace_bytes, stream=None) -> int:
@@ -211,14 +221,15 @@ def attention_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal:
 
 
 def attention_backward(q, k, v, o, lse, dO, causal: bool = False, scale: Optional[float] = None,
-                       workspace: Optional[torch.Tensor] = None):
-    """dQ, dK, dV for bf16 [B, N, H, d] CUDA tensors."""
+                       workspace: Optional[torch.Tensor] = None, deterministic: bool = False):
+    """dQ, dK, dV for bf16 [B, N, H, d] CUDA tensors (fa_bwd, or fa_bwd_deterministic)."""
     B, N, H, d = _shape(q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     nbytes = fa_bwd_workspace_bytes(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(nbytes, device=q.device, dtype=torch.uint8)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    _check("fa_bwd", fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale,
-                            workspace, workspace.numel() * workspace.element_size()))
+    fn = fa_bwd_deterministic if deterministic else fa_bwd
+    _check(fn.__name__, fn(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale,
+                           workspace, workspace.numel() * workspace.element_size()))
     return dq, dk, dv

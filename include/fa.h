@@ -79,6 +79,17 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            int B, int H, int N, int d, int causal, float scale,
            void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bitwise-repeatable backward pass: same arguments, workspace and results as fa_bwd (within
+ * the same tolerance of the exact gradients), but every output is accumulated in a fixed
+ * order, so repeated calls on the same inputs give identical bits.  dQ comes from a separate
+ * per-query-tile kernel that recomputes S and dP (1.4x the tensor work of fa_bwd) instead of
+ * fp32 reductions whose arrival order varies.  The pages call the method "exact and
+ * deterministic" ("FlashAttention-2 — FlashAttention-2", section パフォーマンス). */
+int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                         int B, int H, int N, int d, int causal, float scale,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
 /* The three stages fa_bwd runs, exposed so a caller can time or schedule them apart.
  * Calling them in this order on one stream with the same workspace is exactly fa_bwd.
  *  fa_bwd_preprocess: D = rowsum(dO o O) and lse*log2(e) into the workspace; clears the

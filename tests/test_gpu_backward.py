@@ -91,3 +91,42 @@ def test_backward_full_head_at_4k(fa):
                                 w.scale, True)
     for name, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), refs):
         assert rel_l2(to_np(g[b, :, h]), r) <= GRAD_REL_L2, name
+
+
+# ------------------------------------------------------------------ deterministic variant
+
+@pytest.mark.parametrize("B,N,H,d", [(2, 1000, 3, 128), (3, 300, 2, 64), (1, 1, 1, 64),
+                                     (1, 129, 1, 128), (1, 640, 4, 64)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_deterministic_backward_parity(fa, B, N, H, d, causal):
+    t = synthetic.draw(B, N, H, d, 3000 + N + d, "bf16", with_grad=True)
+    scale = 1.0 / math.sqrt(d)
+    q, k, v, dO = cuda(t, ("q", "k", "v", "dO"))
+    o, lse = fa.attention_forward(q, k, v, causal=causal, scale=scale)
+    got = fa.attention_backward(q, k, v, o, lse, dO, causal=causal, scale=scale, deterministic=True)
+    torch.cuda.synchronize()
+    assert fa.fa_read_device_status() == 0
+    refs = oracle.backward(*(synthetic.to_f64(t[n]) for n in ("q", "k", "v", "dO")), scale, causal)
+    for name, g, r in zip(("dq", "dk", "dv"), got, refs):
+        assert grad_err(to_np(g), r) <= GRAD_REL_L2, (name, grad_err(to_np(g), r))
+
+
+@pytest.mark.parametrize("w", [synthetic.fwdbwd(4096), synthetic.long_context()], ids=lambda w: w.label())
+def test_deterministic_backward_is_bitwise_repeatable_at_full_size(fa, w):
+    t = synthetic.draw_workload(w, with_grad=True)
+    q, k, v, dO = cuda(t, ("q", "k", "v", "dO"))
+    o, lse = fa.attention_forward(q, k, v, causal=w.causal, scale=w.scale)
+    a = fa.attention_backward(q, k, v, o, lse, dO, causal=w.causal, scale=w.scale, deterministic=True)
+    b = fa.attention_backward(q, k, v, o, lse, dO, causal=w.causal, scale=w.scale, deterministic=True)
+    c = fa.attention_backward(q, k, v, o, lse, dO, causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    # and it agrees with the atomic-reduction variant within the gradient tolerance
+    for x, y in zip(a, c):
+        assert rel_l2(to_np(x), to_np(y)) <= 2e-3
+    rng = np.random.default_rng(w.seed)
+    rows = np.unique(rng.integers(0, w.N, 32))
+    Q, K, V, DO = (synthetic.to_f64(t[n][0, :, 0]) for n in ("q", "k", "v", "dO"))
+    ref = oracle.dq_rows(Q, K, V, DO, w.scale, w.causal, rows)
+    assert rel_l2(to_np(a[0][0, rows, 0]), ref) <= GRAD_REL_L2
