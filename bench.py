@@ -471,6 +471,27 @@ def run_sweep(path: str, reps: int = 20, warmup: int = 3):
                 del dO, dq, dk, dv, ws
             del q, k, v, o, lse, t
             torch.cuda.empty_cache()
+        # Decoding (split-KV): HBM-bound, reported against the measured copy bandwidth.
+        for name, B, Nq, Nk, H, d, seed in synthetic.decode_workloads():
+            t = synthetic.draw_decode(B, Nq, Nk, H, d, seed, "bf16")
+            q, k, v = (t[n].to(dev) for n in ("q", "k", "v"))
+            o = torch.empty_like(q)
+            lse = torch.empty((B, H, Nq), device=dev, dtype=torch.float32)
+            nb = fa.fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d)
+            ws = torch.empty(nb, device=dev, dtype=torch.uint8)
+            dec = lambda: fa.fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, 1, 1.0 / math.sqrt(d),
+                                            fa.FA_DTYPE_BF16, ws, nb, stream)
+            assert dec() == 0
+            med, best = timed(dec)
+            kv_bytes = 2 * B * Nk * H * d * 2
+            rec = {"workload": f"{name}:B{B}xNq{Nq}xNk{Nk}xH{H}xd{d}-causal-bf16", "pass": "fwd_splitkv",
+                   "ms": round(med, 4), "ms_best": round(best, 4),
+                   "kv_gbs": round(kv_bytes / (med * 1e-3) / 1e9, 1),
+                   "frac_of_hbm": round(kv_bytes / (med * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_src}
+            out.write(json.dumps(rec) + "\n")
+            print(json.dumps(rec), file=sys.stderr)
+            del q, k, v, o, lse, ws, t
+            torch.cuda.empty_cache()
     if fa.fa_read_device_status(stream) != 0:
         raise RuntimeError("device status word reports a timeout")
 

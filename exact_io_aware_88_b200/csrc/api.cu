@@ -7,6 +7,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "fa.h"
@@ -80,7 +81,8 @@ int check_shape(int B, int H, int N, int d, float scale) {
 
 // 4-D view [B][N][H][d] (innermost first: d, H, N, B) of a bf16 tensor, tiled in boxes of
 // 64 d-elements (128 bytes, the 128-byte swizzle span) x 1 head x 128 rows x 1 batch.
-int encode_bnhd(CUtensorMap* m, const void* ptr, int B, int N, int H, int d) {
+int encode_bnhd(CUtensorMap* m, const void* ptr, int B, int N, int H, int d,
+                CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2,
@@ -88,7 +90,7 @@ int encode_bnhd(CUtensorMap* m, const void* ptr, int B, int N, int H, int d) {
                                  static_cast<cuuint64_t>(N) * H * d * 2};
   const cuuint32_t box[4] = {64, 1, 128, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims,
+  CUresult r = g_encode(m, dt, 4, const_cast<void*>(ptr), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -102,6 +104,30 @@ int from_cuda(cudaError_t e) {
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Split-KV plan: enough (query tile, key slice) units to give every SM of a B200 two (296),
+// at most 64 slices, never more slices than key tiles.  Device-independent, so the
+// workspace size depends on the problem only.
+constexpr long long kSplitTargetUnits = 296;
+void splitkv_plan(int B, int H, int Nq, int Nk, int* n_split, int* tiles_per_split) {
+  const long long kv_tiles = (Nk + 127) / 128;
+  const long long base = static_cast<long long>(B) * H * ((Nq + 127) / 128);
+  long long n = (kSplitTargetUnits + base - 1) / base;
+  n = std::max(1LL, std::min(n, std::min(kv_tiles, 64LL)));
+  const long long tps = (kv_tiles + n - 1) / n;
+  *tiles_per_split = static_cast<int>(tps);
+  *n_split = static_cast<int>((kv_tiles + tps - 1) / tps);
+}
+
+int check_splitkv(int B, int H, int Nq, int Nk, int d, int causal, float scale) {
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || !isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (causal && Nq > Nk) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long double>(B) * std::max(Nq, Nk) * H * d > 9.0e15L) return FA_ERR_INVALID_ARG;
+  const long long units = static_cast<long long>(B) * H * ((Nq + 127) / 128) * 64;
+  if (units > 0x7fffffffLL || Nk > 0x7fffff80) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
 
 }  // namespace
 
@@ -323,6 +349,54 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   if ((rc = from_cuda(fa::launch_bwd_pre(a, st)))) return rc;
   if ((rc = from_cuda(fa::launch_bwd_main(a, st, true)))) return rc;
   return from_cuda(fa::launch_bwd_convert(a, st));
+}
+
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d) {
+  if (check_splitkv(B, H, Nq, Nk, d, 0, 1.0f) != FA_OK) return 0;
+  int n_split = 1, tps = 1;
+  splitkv_plan(B, H, Nq, Nk, &n_split, &tps);
+  const size_t rows = static_cast<size_t>(n_split) * B * H * Nq;
+  return round_up(rows * d * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
+}
+
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                   int Nq, int Nk, int d, int causal, float scale, int dtype, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  int rc = check_splitkv(B, H, Nq, Nk, d, causal, scale);
+  if (rc) return rc;
+  if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_FP16) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_MISALIGNED;
+  const size_t need = fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d);
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  fa::SplitKvArgs a;
+  const CUtensorMapDataType dt =
+      dtype == FA_DTYPE_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if ((rc = encode_bnhd(&a.tm_q, q, B, Nq, H, d, dt)) ||
+      (rc = encode_bnhd(&a.tm_k, k, B, Nk, H, d, dt)) ||
+      (rc = encode_bnhd(&a.tm_v, v, B, Nk, H, d, dt)))
+    return rc;
+  splitkv_plan(B, H, Nq, Nk, &a.n_split, &a.tiles_per_split);
+  const size_t rows = static_cast<size_t>(a.n_split) * B * H * Nq;
+  char* ws = static_cast<char*>(workspace);
+  a.part_o = reinterpret_cast<float*>(ws);
+  a.part_lse = reinterpret_cast<float*>(ws + round_up(rows * d * sizeof(float), 256));
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.H = H;
+  a.Nq = Nq;
+  a.Nk = Nk;
+  a.d = d;
+  a.causal = causal ? 1 : 0;
+  a.f16 = dtype == FA_DTYPE_FP16 ? 1 : 0;
+  a.scale = scale;
+  a.status = di.status;
+  return from_cuda(fa::launch_fwd_splitkv(a, static_cast<cudaStream_t>(stream)));
 }
 
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H,

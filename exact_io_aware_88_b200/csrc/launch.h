@@ -37,7 +37,20 @@ struct BwdArgs {
   int num_sms;
 };
 
+struct SplitKvArgs {
+  CUtensorMap tm_q, tm_k, tm_v;  // q over [B][Nq][H][d]; k, v over [B][Nk][H][d]
+  void* o;                       // [B][Nq][H][d] bf16 or fp16
+  float* lse;                    // [B][H][Nq]
+  float* part_o;                 // [n_split][B*H][Nq][d] fp32 workspace
+  float* part_lse;               // [n_split][B*H][Nq] fp32 workspace
+  int B, H, Nq, Nk, d, causal, f16;
+  int n_split, tiles_per_split;
+  float scale;
+  int* status;
+};
+
 cudaError_t launch_fwd_sm100(const FwdArgs& a, cudaStream_t s);
+cudaError_t launch_fwd_splitkv(const SplitKvArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_pre(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t s, bool with_dq);
 cudaError_t launch_bwd_dq(const BwdArgs& a, cudaStream_t s);

@@ -27,6 +27,8 @@ FA_ERR_MISALIGNED = 3
 FA_ERR_WORKSPACE = 4
 FA_ERR_CUDA = 5
 FA_ERR_TIMEOUT = 6
+FA_DTYPE_BF16 = 0
+FA_DTYPE_FP16 = 1
 
 
 class FAError(RuntimeError):
@@ -65,6 +67,10 @@ _lib.fa_bwd_dq_convert.argtypes = [_P, _I, _I, _I, _I, _F, _P, _SZ, _P]
 _lib.fa_bwd_dq_convert.restype = _I
 _lib.fa_bwd_noalloc.argtypes = [_P] * 9 + [_I, _I, _I, _I, _I, _F, _P]
 _lib.fa_bwd_noalloc.restype = _I
+_lib.fa_fwd_splitkv_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
+_lib.fa_fwd_splitkv_workspace_bytes.restype = _SZ
+_lib.fa_fwd_splitkv.argtypes = [_P] * 5 + [_I] * 6 + [_F, _I, _P, _SZ, _P]
+_lib.fa_fwd_splitkv.restype = _I
 _lib.fa_fwd_f32.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.fa_fwd_f32.restype = _I
 _lib.fa_read_device_status.argtypes = [ctypes.POINTER(_I), _P]
@@ -82,7 +88,8 @@ _lib.fa_debug_wait_timeout.restype = _I
 
 # Every symbol the C headers declare, for the ABI self-check.
 EXPORTED = sorted(["fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess", "fa_bwd_kv",
-                   "fa_bwd_dq_convert", "fa_bwd_noalloc", "fa_fwd_f32", "fa_read_device_status", "fa_status_string",
+                   "fa_bwd_dq_convert", "fa_bwd_noalloc", "fa_fwd_f32", "fa_fwd_splitkv",
+                   "fa_fwd_splitkv_workspace_bytes", "fa_read_device_status", "fa_status_string",
                    "fa_version", "fa_debug_umma_tile", "fa_debug_wait_timeout",
                    "fa_debug_exp2"])
 
@@ -165,6 +172,17 @@ def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, s
                                _stream(stream))
 
 
+def fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d) -> int:
+    return _lib.fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d)
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, dtype, workspace,
+                   workspace_bytes, stream=None) -> int:
+    return _lib.fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
+                               int(causal), float(scale), int(dtype), _ptr(workspace),
+                               int(workspace_bytes), _stream(stream))
+
+
 def fa_fwd_f32(q, k, v, o, lse, B, H, N, d, causal, scale, stream=None) -> int:
     return _lib.fa_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
                            int(causal), float(scale), _stream(stream))
@@ -233,3 +251,21 @@ def attention_backward(q, k, v, o, lse, dO, causal: bool = False, scale: Optiona
     _check(fn.__name__, fn(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale,
                            workspace, workspace.numel() * workspace.element_size()))
     return dq, dk, dv
+
+
+def attention_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True,
+                     scale: Optional[float] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """O, LSE for q [B, Nq, H, d] against k, v [B, Nk, H, d] (bf16 or fp16), split-KV."""
+    B, Nq, H, d = _shape(q)
+    Nk = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dt = {torch.bfloat16: FA_DTYPE_BF16, torch.float16: FA_DTYPE_FP16}.get(q.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), device=q.device, dtype=torch.float32)
+    nb = fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d)
+    ws = torch.empty(max(nb, 256), device=q.device, dtype=torch.uint8)
+    _check("fa_fwd_splitkv", fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, dt,
+                                            ws, ws.numel()))
+    return o, lse

@@ -131,6 +131,25 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    const void* dO, void* dq, void* dk, void* dv,
                    int B, int H, int N, int d, int causal, float scale, void* stream);
 
+/* Element types of fa_fwd_splitkv. */
+enum { FA_DTYPE_BF16 = 0, FA_DTYPE_FP16 = 1 };
+
+/* Forward pass for few queries against many keys (decoding), with the key sequence split
+ * across CTAs and the slices merged exactly through their logsumexps.  Prefill and decode
+ * are measured separately ("FlashAttention-2を読む", section 実装上の差を検証可能な形で残す);
+ * fp16 is FA-2's other input type ("Flash Attention 2で打破するローカルLLMの「メモリの壁」",
+ * section Hugging Face Transformersでの有効化設定).
+ *   q : [B][Nq][H][d]; k, v : [B][Nk][H][d]; o : [B][Nq][H][d]  (all bf16 or all fp16,
+ *   `dtype` = FA_DTYPE_BF16 / FA_DTYPE_FP16);  lse : [B][H][Nq] fp32.
+ *   Causal: the last query is aligned with the last key -- query i sees keys
+ *   j <= i + Nk - Nq; requires Nq <= Nk.  Non-causal: any Nq, Nk >= 1.  d in {64, 128}.
+ *   workspace: caller-owned device memory, >= fa_fwd_splitkv_workspace_bytes(...), 256-byte
+ *   aligned (fp32 partial outputs and logsumexps of every slice). */
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d);
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int H, int Nq, int Nk, int d, int causal, float scale, int dtype,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
 /* Forward pass in fp32 on the CUDA cores (no tensor cores, no TF32), for fp32 inputs.
  *   q, k, v, o : [B][N][H][d] fp32; lse : [B][H][N] fp32.  1 <= d <= 128, d % 4 == 0. */
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,

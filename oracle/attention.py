@@ -39,11 +39,13 @@ import numpy as np
 DEFAULT_SLAB = 1024
 
 
-def _mask_rows(S: np.ndarray, rows: np.ndarray, causal: bool) -> np.ndarray:
-    """Set S[r, j] = -inf where key j is not visible to query rows[r]."""
+def _mask_rows(S: np.ndarray, rows: np.ndarray, causal: bool, offset: int = 0) -> np.ndarray:
+    """Set S[r, j] = -inf where key j is not visible to query rows[r]: under the causal mask
+    query i sees keys j <= i + offset (offset = Nk - Nq aligns the last query with the last
+    key when there are fewer queries than keys; 0 for square problems)."""
     if causal:
         cols = np.arange(S.shape[1])
-        S = np.where(cols[None, :] <= rows[:, None], S, -np.inf)
+        S = np.where(cols[None, :] <= rows[:, None] + offset, S, -np.inf)
     return S
 
 
@@ -61,17 +63,20 @@ def _softmax_rows(S: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
 
 def forward_head(Q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float, causal: bool,
                  slab: int = DEFAULT_SLAB) -> Tuple[np.ndarray, np.ndarray]:
-    """One (batch, head): Q, K, V are [N, d].  Returns O [N, d] and LSE [N]."""
+    """One (batch, head): Q is [Nq, d], K and V are [Nk, d] (Nq = Nk for the square problems
+    of the main path; Nq <= Nk for decoding, where the causal mask is aligned to the last
+    key: query i sees keys j <= i + Nk - Nq).  Returns O [Nq, d] and LSE [Nq]."""
     Q = np.asarray(Q, np.float64)
     K = np.asarray(K, np.float64)
     V = np.asarray(V, np.float64)
     N = Q.shape[0]
+    offset = K.shape[0] - N
     O = np.empty((N, V.shape[1]), np.float64)
     lse = np.empty(N, np.float64)
     for r0 in range(0, N, slab):
         rows = np.arange(r0, min(N, r0 + slab))
         S = scale * (Q[rows] @ K.T)              # step 1: S = scale * Q K^T
-        S = _mask_rows(S, rows, causal)
+        S = _mask_rows(S, rows, causal, offset)
         P, lse[rows] = _softmax_rows(S)          # step 2: P = softmax(S)
         O[rows] = P @ V                          # step 3: O = P V
     return O, lse
@@ -110,9 +115,9 @@ def _heads(x: np.ndarray):
 
 
 def forward(q, k, v, scale: float, causal: bool, heads: Optional[Sequence[Tuple[int, int]]] = None):
-    """[B, N, H, d] inputs.  Returns O [B, N, H, d] and LSE [B, H, N] (float64).
-
-    ``heads`` restricts the work to the listed (b, h) pairs; other entries stay NaN.
+    """q [B, Nq, H, d], k and v [B, Nk, H, d].  Returns O [B, Nq, H, d] and LSE [B, H, Nq]
+    (float64).  ``heads`` restricts the work to the listed (b, h) pairs; other entries stay
+    NaN.
     """
     q = np.asarray(q, np.float64)
     B, N, H, _ = q.shape

@@ -101,6 +101,8 @@ def draw(B: int, N: int, H: int, d: int, seed: int, dtype: str = "bf16",
         t = torch.randn((B, N, H, d), generator=g, dtype=torch.float32)
         if dtype == "bf16":
             t = t.to(torch.bfloat16)
+        elif dtype == "f16":
+            t = t.to(torch.float16)
         elif dtype != "f32":
             raise ValueError(f"unknown dtype {dtype}")
         out[nm] = t.contiguous()
@@ -115,3 +117,27 @@ def draw_workload(w: Workload, with_grad: Optional[bool] = None) -> Dict[str, to
 def to_f64(t: torch.Tensor):
     """Exact upcast of a bf16/fp32 tensor to a float64 numpy array."""
     return t.to(torch.float64).numpy()
+
+
+def draw_decode(B: int, Nq: int, Nk: int, H: int, d: int, seed: int, dtype: str = "bf16"
+                ) -> Dict[str, torch.Tensor]:
+    """q [B, Nq, H, d] and k, v [B, Nk, H, d] for decoding workloads (q drawn first)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    out = {}
+    for nm, n in (("q", Nq), ("k", Nk), ("v", Nk)):
+        t = torch.randn((B, n, H, d), generator=g, dtype=torch.float32)
+        t = t.to({"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[dtype])
+        out[nm] = t.contiguous()
+    return out
+
+
+def decode_workloads():
+    """Decoding shapes (not among the pages' prefill sweep): a batch of 8 sequences, 16 heads
+    of dim 128, one new query token (and 16 for speculative-style multi-token steps) against
+    4k / 16k / 64k cached keys, causal, bf16.  Returns (name, B, Nq, Nk, H, d, seed)."""
+    out = []
+    for Nq in (1, 16):
+        for Nk in (4096, 16384, 65536):
+            out.append((f"decode_q{Nq}_k{Nk}", 8, Nq, Nk, 16, 128, 1005))
+    return out

@@ -1,0 +1,83 @@
+"""GPU parity of the split-KV (decoding) forward against the fp64 oracle, bf16 and fp16."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from tests._helpers import LSE_MAX_ABS, O_MAX_ABS, O_REL_L2, max_abs, rel_l2, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fa():
+    import __graft_entry__
+    __graft_entry__.build()
+    from exact_io_aware_88_b200 import fa as mod
+    assert torch.cuda.is_available()
+    return mod
+
+
+def _case(fa, B, Nq, Nk, H, d, causal, dtype, seed):
+    t = synthetic.draw_decode(B, Nq, Nk, H, d, seed, dtype)
+    q, k, v = (t[n].cuda() for n in ("q", "k", "v"))
+    scale = 1.0 / math.sqrt(d)
+    o, lse = fa.attention_decode(q, k, v, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.fa_read_device_status() == 0
+    O_ref, L_ref = oracle.forward(*(synthetic.to_f64(t[n]) for n in ("q", "k", "v")), scale, causal)
+    return to_np(o), to_np(lse), O_ref, L_ref
+
+
+@pytest.mark.parametrize("B,Nq,Nk,H,d", [
+    (2, 1, 1, 3, 64), (2, 1, 300, 3, 128), (1, 4, 1000, 2, 128), (2, 37, 700, 2, 64),
+    (1, 128, 2048, 4, 128), (1, 200, 1000, 2, 128), (1, 100, 100, 2, 64), (3, 16, 4096, 2, 64),
+])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_splitkv_parity(fa, B, Nq, Nk, H, d, causal, dtype):
+    O, L, O_ref, L_ref = _case(fa, B, Nq, Nk, H, d, causal, dtype, 4000 + Nq + Nk + d)
+    assert max_abs(O, O_ref) <= O_MAX_ABS, max_abs(O, O_ref)
+    assert rel_l2(O, O_ref) <= O_REL_L2, rel_l2(O, O_ref)
+    assert max_abs(L, L_ref) <= LSE_MAX_ABS, max_abs(L, L_ref)
+
+
+def test_splitkv_square_causal_matches_forward_kernel(fa):
+    # Nq = Nk: the bottom-right causal alignment coincides with the square mask of fa_fwd.
+    t = synthetic.draw(2, 640, 3, 128, 77, "bf16")
+    q, k, v = (t[n].cuda() for n in ("q", "k", "v"))
+    o1, l1 = fa.attention_forward(q, k, v, causal=True)
+    o2, l2 = fa.attention_decode(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert max_abs(to_np(o1), to_np(o2)) <= 8e-3
+    assert max_abs(to_np(l1), to_np(l2)) <= 1e-4
+
+
+@pytest.mark.parametrize("Nk", [16384, 65536])
+def test_splitkv_decode_one_token_full_size(fa, Nk):
+    B, Nq, H, d = 8, 1, 16, 128
+    O, L, O_ref, L_ref = None, None, None, None
+    t = synthetic.draw_decode(B, Nq, Nk, H, d, 5000 + Nk, "bf16")
+    q, k, v = (t[n].cuda() for n in ("q", "k", "v"))
+    o, lse = fa.attention_decode(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    for b, h in [(0, 0), (B - 1, H - 1), (3, 7)]:
+        Q, K, V = (synthetic.to_f64(t[n][b, :, h]) for n in ("q", "k", "v"))
+        Or, Lr = oracle.forward_head(Q, K, V, 1.0 / math.sqrt(d), True)
+        assert max_abs(to_np(o[b, :, h]), Or) <= O_MAX_ABS
+        assert abs(float(lse[b, h, 0]) - Lr[0]) <= LSE_MAX_ABS
+
+
+def test_splitkv_rejects_bad_arguments(fa):
+    a16 = 1 << 20
+    p = [a16] * 5
+    nb = fa.fa_fwd_splitkv_workspace_bytes(1, 1, 4, 100, 128)
+    assert nb > 0
+    # causal needs Nq <= Nk
+    assert fa.fa_fwd_splitkv(*p, 1, 1, 200, 100, 128, 1, 0.1, 0, a16, 1 << 30, stream=0) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_fwd_splitkv(*p, 1, 1, 4, 100, 96, 0, 0.1, 0, a16, 1 << 30, stream=0) == fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_fwd_splitkv(*p, 1, 1, 4, 100, 128, 0, 0.1, 7, a16, 1 << 30, stream=0) == fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_fwd_splitkv(*p, 1, 1, 4, 100, 128, 0, 0.1, 0, a16, nb - 1, stream=0) == fa.FA_ERR_WORKSPACE

@@ -275,3 +275,50 @@ def test_slab_size_does_not_change_results():
         gb = backward_head(Q, K, V, dO, 0.5, causal, slab=7)
         for x, y in zip(ga, gb):
             np.testing.assert_allclose(x, y, atol=1e-12)
+
+
+# ---------------------------------------------------------------- fewer queries than keys
+
+def test_single_last_query_sees_every_key():
+    # Decoding one token: with the causal mask aligned to the last key, the only query sees
+    # all keys, i.e. it equals the non-causal result.
+    Nk, d = 57, 6
+    Q, K, V = rnd(90, 1, d), rnd(91, Nk, d), rnd(92, Nk, d)
+    Oc, lc = forward_head(Q, K, V, 0.4, True)
+    On, ln = forward_head(Q, K, V, 0.4, False)
+    np.testing.assert_allclose(Oc, On, atol=1e-14)
+    np.testing.assert_allclose(lc, ln, atol=1e-14)
+
+
+def test_bottom_right_causal_row_equals_noncausal_over_its_visible_keys():
+    Nq, Nk, d = 9, 40, 5
+    Q, K, V = rnd(93, Nq, d), rnd(94, Nk, d), rnd(95, Nk, d)
+    O, l = forward_head(Q, K, V, 0.7, True)
+    for i in range(Nq):
+        vis = i + Nk - Nq + 1
+        Op, lp = forward_head(Q[i:i + 1], K[:vis], V[:vis], 0.7, False)
+        np.testing.assert_allclose(O[i], Op[0], atol=1e-14)
+        assert abs(l[i] - lp[0]) < 1e-13
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_split_merge_rule(causal):
+    # Splitting the keys, attending to each part and merging with the logsumexp rule
+    # (O = sum_s exp(L_s - L) O_s, L = log sum_s exp L_s) reproduces attention over all keys.
+    Nq, Nk, d = 7, 61, 8
+    Q, K, V = rnd(96, Nq, d), rnd(97, Nk, d), rnd(98, Nk, d)
+    O, L = forward_head(Q, K, V, 0.3, causal)
+    off = Nk - Nq
+    parts = []
+    for a, b in [(0, 20), (20, 47), (47, Nk)]:
+        S = 0.3 * Q @ K[a:b].T
+        if causal:
+            S = np.where(np.arange(a, b)[None, :] <= np.arange(Nq)[:, None] + off, S, -np.inf)
+        m = S.max(axis=1)
+        E = np.exp(S - m[:, None])
+        parts.append((E @ V[a:b] / E.sum(1)[:, None], m + np.log(E.sum(1))))
+    Ls = np.stack([p[1] for p in parts])
+    Lm = np.log(np.exp(Ls - Ls.max(0)).sum(0)) + Ls.max(0)
+    Om = sum(np.exp(p[1] - Lm)[:, None] * p[0] for p in parts)
+    np.testing.assert_allclose(Om, O, atol=1e-13)
+    np.testing.assert_allclose(Lm, L, atol=1e-13)
