@@ -43,6 +43,7 @@ struct SplitKvArgs {
   float* lse;                    // [B][H][Nq]
   float* part_o;                 // [n_split][B*H][Nq][d] fp32 workspace
   float* part_lse;               // [n_split][B*H][Nq] fp32 workspace
+  const uint8_t* block_mask;     // block-sparse: [ceil(Nq/128)][ceil(Nk/128)] or null
   int B, H, Nq, Nk, d, causal, f16;
   int n_split, tiles_per_split;
   float scale;

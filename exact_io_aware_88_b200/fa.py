@@ -71,6 +71,10 @@ _lib.fa_fwd_splitkv_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
 _lib.fa_fwd_splitkv_workspace_bytes.restype = _SZ
 _lib.fa_fwd_splitkv.argtypes = [_P] * 5 + [_I] * 6 + [_F, _I, _P, _SZ, _P]
 _lib.fa_fwd_splitkv.restype = _I
+_lib.fa_fwd_block_sparse_workspace_bytes.argtypes = [_I, _I, _I, _I]
+_lib.fa_fwd_block_sparse_workspace_bytes.restype = _SZ
+_lib.fa_fwd_block_sparse.argtypes = [_P] * 5 + [_I] * 5 + [_F, _P, _P, _SZ, _P]
+_lib.fa_fwd_block_sparse.restype = _I
 _lib.fa_fwd_f32.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.fa_fwd_f32.restype = _I
 _lib.fa_read_device_status.argtypes = [ctypes.POINTER(_I), _P]
@@ -89,7 +93,8 @@ _lib.fa_debug_wait_timeout.restype = _I
 # Every symbol the C headers declare, for the ABI self-check.
 EXPORTED = sorted(["fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess", "fa_bwd_kv",
                    "fa_bwd_dq_convert", "fa_bwd_noalloc", "fa_fwd_f32", "fa_fwd_splitkv",
-                   "fa_fwd_splitkv_workspace_bytes", "fa_read_device_status", "fa_status_string",
+                   "fa_fwd_splitkv_workspace_bytes", "fa_fwd_block_sparse",
+                   "fa_fwd_block_sparse_workspace_bytes", "fa_read_device_status", "fa_status_string",
                    "fa_version", "fa_debug_umma_tile", "fa_debug_wait_timeout",
                    "fa_debug_exp2"])
 
@@ -183,6 +188,17 @@ def fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, dtype, works
                                int(workspace_bytes), _stream(stream))
 
 
+def fa_fwd_block_sparse_workspace_bytes(B, H, N, d) -> int:
+    return _lib.fa_fwd_block_sparse_workspace_bytes(B, H, N, d)
+
+
+def fa_fwd_block_sparse(q, k, v, o, lse, B, H, N, d, causal, scale, block_mask, workspace,
+                        workspace_bytes, stream=None) -> int:
+    return _lib.fa_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                                    int(causal), float(scale), _ptr(block_mask), _ptr(workspace),
+                                    int(workspace_bytes), _stream(stream))
+
+
 def fa_fwd_f32(q, k, v, o, lse, B, H, N, d, causal, scale, stream=None) -> int:
     return _lib.fa_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
                            int(causal), float(scale), _stream(stream))
@@ -268,4 +284,19 @@ def attention_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: 
     ws = torch.empty(max(nb, 256), device=q.device, dtype=torch.uint8)
     _check("fa_fwd_splitkv", fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, dt,
                                             ws, ws.numel()))
+    return o, lse
+
+
+def attention_block_sparse(q, k, v, block_mask: torch.Tensor, causal: bool = False,
+                           scale: Optional[float] = None):
+    """O, LSE for bf16 [B, N, H, d] tensors with a [ceil(N/128), ceil(N/128)] uint8 mask."""
+    B, N, H, d = _shape(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    m = block_mask.to(device=q.device, dtype=torch.uint8).contiguous()
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    nb = fa_fwd_block_sparse_workspace_bytes(B, H, N, d)
+    ws = torch.empty(max(nb, 256), device=q.device, dtype=torch.uint8)
+    _check("fa_fwd_block_sparse", fa_fwd_block_sparse(q, k, v, o, lse, B, H, N, d, causal, scale,
+                                                      m, ws, ws.numel()))
     return o, lse

@@ -150,6 +150,21 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
                    int B, int H, int Nq, int Nk, int d, int causal, float scale, int dtype,
                    void* workspace, size_t workspace_bytes, void* stream);
 
+/* Block-sparse forward pass, the extension described with the original method
+ * ("FlashAttention――GPUメモリの読み書きを減らし、注意機構を正確なまま高速・省メモリに",
+ * section 手法): key j is visible to query i iff block_mask[i/128][j/128] != 0 (and, if
+ * causal, j <= i); masked 128x128 blocks are neither loaded nor computed.
+ *   q, k, v, o : [B][N][H][d] bf16; lse : [B][H][N] fp32; d in {64, 128}; N <= 131072.
+ *   block_mask : DEVICE pointer, [ceil(N/128)][ceil(N/128)] bytes, shared by all batches and
+ *                heads.
+ *   A query that sees no key at all gets O = 0 and lse = -inf.
+ *   workspace : >= fa_fwd_block_sparse_workspace_bytes(B, H, N, d), 256-byte aligned. */
+size_t fa_fwd_block_sparse_workspace_bytes(int B, int H, int N, int d);
+int fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int H, int N, int d, int causal, float scale,
+                        const uint8_t* block_mask, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
 /* Forward pass in fp32 on the CUDA cores (no tensor cores, no TF32), for fp32 inputs.
  *   q, k, v, o : [B][N][H][d] fp32; lse : [B][H][N] fp32.  1 <= d <= 128, d % 4 == 0. */
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,

@@ -7,5 +7,5 @@ passage of the source pages each step follows.
 """
 from .attention import (  # noqa: F401
     forward, backward, forward_head, backward_head,
-    forward_rows, dq_rows, kv_grad_tail, scalar_loop_head,
+    forward_rows, dq_rows, kv_grad_tail, scalar_loop_head, forward_head_block_sparse,
 )

@@ -228,3 +228,32 @@ def scalar_loop_head(Q, K, V, dO, scale: float, causal: bool):
                 dQ[i][t] += scale * dS * K[j][t]
                 dK[j][t] += scale * dS * Q[i][t]
     return O, LSE, dQ, dK, dV
+
+
+# ----------------------------------------------------------------------------------------
+# Block-sparse attention: the FlashAttention summary's extension ("FlashAttention――GPUメモリ
+# の読み書きを減らし、注意機構を正確なまま高速・省メモリに", section 手法): whole blocks of S are
+# skipped.  Key j is visible to query i iff block_mask[i // bq, j // bk] is set (and, under the
+# causal mask, j <= i).  A query that sees no key at all gets O = 0 and LSE = -inf (the
+# empty sum): the pages leave that case open.
+# ----------------------------------------------------------------------------------------
+
+def forward_head_block_sparse(Q, K, V, scale: float, causal: bool, block_mask, bq: int = 128,
+                              bk: int = 128):
+    """Q, K, V [N, d]; block_mask [ceil(N/bq), ceil(N/bk)] of 0/1.  Returns O [N, d], LSE [N]."""
+    Q = np.asarray(Q, np.float64)
+    K = np.asarray(K, np.float64)
+    V = np.asarray(V, np.float64)
+    N = Q.shape[0]
+    mask = np.asarray(block_mask).astype(bool)
+    vis = np.repeat(np.repeat(mask, bq, axis=0), bk, axis=1)[:N, :K.shape[0]]
+    if causal:
+        vis &= np.arange(K.shape[0])[None, :] <= np.arange(N)[:, None]
+    S = np.where(vis, scale * (Q @ K.T), -np.inf)
+    O = np.zeros((N, V.shape[1]))
+    lse = np.full(N, -np.inf)
+    live = vis.any(axis=1)
+    if live.any():
+        P, lse[live] = _softmax_rows(S[live])
+        O[live] = P @ V
+    return O, lse

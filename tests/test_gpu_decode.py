@@ -81,3 +81,42 @@ def test_splitkv_rejects_bad_arguments(fa):
     assert fa.fa_fwd_splitkv(*p, 1, 1, 4, 100, 96, 0, 0.1, 0, a16, 1 << 30, stream=0) == fa.FA_ERR_UNSUPPORTED
     assert fa.fa_fwd_splitkv(*p, 1, 1, 4, 100, 128, 0, 0.1, 7, a16, 1 << 30, stream=0) == fa.FA_ERR_UNSUPPORTED
     assert fa.fa_fwd_splitkv(*p, 1, 1, 4, 100, 128, 0, 0.1, 0, a16, nb - 1, stream=0) == fa.FA_ERR_WORKSPACE
+
+
+# ------------------------------------------------------------------ block-sparse forward
+
+def _bs_case(fa, B, N, H, d, causal, mask, seed):
+    t = synthetic.draw(B, N, H, d, seed, "bf16")
+    q, k, v = (t[n].cuda() for n in ("q", "k", "v"))
+    scale = 1.0 / math.sqrt(d)
+    o, lse = fa.attention_block_sparse(q, k, v, torch.from_numpy(mask), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.fa_read_device_status() == 0
+    for b in range(B):
+        for h in range(H):
+            Or, Lr = oracle.forward_head_block_sparse(*(synthetic.to_f64(t[n][b, :, h]) for n in ("q", "k", "v")),
+                                                      scale, causal, mask)
+            O, L = to_np(o[b, :, h]), to_np(lse[b, h])
+            assert max_abs(O, Or) <= O_MAX_ABS
+            if np.linalg.norm(Or) > 0:
+                assert rel_l2(O, Or) <= O_REL_L2
+            live = np.isfinite(Lr)
+            assert np.all(np.isneginf(L[~live])) and np.all(O[~live] == 0)
+            assert max_abs(L[live], Lr[live]) <= LSE_MAX_ABS
+
+
+@pytest.mark.parametrize("N,d", [(1000, 128), (700, 64), (129, 128)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_sparse_random_masks(fa, N, d, causal):
+    nt = (N + 127) // 128
+    mask = (np.random.default_rng(N + d).random((nt, nt)) < 0.5).astype(np.uint8)
+    mask[0, 0] = 1
+    _bs_case(fa, 2, N, 2, d, causal, mask, 6000 + N)
+
+
+def test_block_sparse_all_ones_equals_dense_and_empty_rows(fa):
+    N, d = 640, 128
+    _bs_case(fa, 1, N, 3, d, True, np.ones((5, 5), np.uint8), 6100)
+    m = np.eye(5, dtype=np.uint8)
+    m[2, 2] = 0  # block row 2 sees nothing: O = 0, lse = -inf
+    _bs_case(fa, 1, N, 2, d, False, m, 6101)

@@ -322,3 +322,45 @@ def test_key_split_merge_rule(causal):
     Om = sum(np.exp(p[1] - Lm)[:, None] * p[0] for p in parts)
     np.testing.assert_allclose(Om, O, atol=1e-13)
     np.testing.assert_allclose(Lm, L, atol=1e-13)
+
+
+# ---------------------------------------------------------------- block-sparse reference
+
+def test_block_sparse_all_ones_is_dense():
+    N, d = 300, 8
+    Q, K, V = rnd(100, N, d), rnd(101, N, d), rnd(102, N, d)
+    m = np.ones((3, 3), np.uint8)
+    for causal in (False, True):
+        O, L = oracle.forward_head_block_sparse(Q, K, V, 0.3, causal, m)
+        Od, Ld = forward_head(Q, K, V, 0.3, causal)
+        np.testing.assert_allclose(O, Od, atol=1e-13)
+        np.testing.assert_allclose(L, Ld, atol=1e-13)
+
+
+def test_block_diagonal_mask_is_independent_blocks():
+    # Only diagonal blocks: each 128-row block attends to itself alone.
+    N, d = 300, 8
+    Q, K, V = rnd(103, N, d), rnd(104, N, d), rnd(105, N, d)
+    O, L = oracle.forward_head_block_sparse(Q, K, V, 0.3, False, np.eye(3, dtype=np.uint8))
+    for a in range(0, N, 128):
+        b = min(N, a + 128)
+        Ob, Lb = forward_head(Q[a:b], K[a:b], V[a:b], 0.3, False)
+        np.testing.assert_allclose(O[a:b], Ob, atol=1e-13)
+        np.testing.assert_allclose(L[a:b], Lb, atol=1e-13)
+
+
+def test_block_sparse_empty_rows_and_brute_force():
+    N, d = 260, 4
+    Q, K, V = rnd(106, N, d), rnd(107, N, d), rnd(108, N, d)
+    m = np.array([[0, 1, 0], [0, 0, 0], [1, 0, 1]], np.uint8)
+    O, L = oracle.forward_head_block_sparse(Q, K, V, 0.5, False, m)
+    assert np.all(O[128:256] == 0) and np.all(np.isneginf(L[128:256]))   # block row 1 is empty
+    for i in (0, 100, 256, 259):                                           # brute force rows
+        keys = [j for j in range(N) if m[i // 128, j // 128]]
+        s = np.array([0.5 * Q[i] @ K[j] for j in keys])
+        p = np.exp(s - s.max()) / np.exp(s - s.max()).sum()
+        np.testing.assert_allclose(O[i], p @ V[keys], atol=1e-13)
+        assert abs(L[i] - (s.max() + np.log(np.exp(s - s.max()).sum()))) < 1e-12
+    # causal: block (0,1) lies above the diagonal, so rows 0..127 see nothing
+    Oc, Lc = oracle.forward_head_block_sparse(Q, K, V, 0.5, True, m)
+    assert np.all(Oc[:128] == 0) and np.all(np.isneginf(Lc[:128]))
