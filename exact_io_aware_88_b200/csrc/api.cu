@@ -71,7 +71,7 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 // Shape checks shared by the bf16 entry points.  Returns FA_OK or an error code.
 int check_shape(int B, int H, int N, int d, float scale) {
-  if (B < 1 || H < 1 || N < 1 || !isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || !(scale > 0.f) || !isfinite(scale)) return FA_ERR_INVALID_ARG;
   const long double elems = static_cast<long double>(B) * N * H * d;
   if (elems > 9.0e15L) return FA_ERR_INVALID_ARG;
   const long long tiles = static_cast<long long>(B) * H * ((N + 127) / 128);
@@ -120,7 +120,8 @@ void splitkv_plan(int B, int H, int Nq, int Nk, int* n_split, int* tiles_per_spl
 }
 
 int check_splitkv(int B, int H, int Nq, int Nk, int d, int causal, float scale) {
-  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || !isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || !(scale > 0.f) || !isfinite(scale))
+    return FA_ERR_INVALID_ARG;
   if (causal && Nq > Nk) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<long double>(B) * std::max(Nq, Nk) * H * d > 9.0e15L) return FA_ERR_INVALID_ARG;
@@ -445,7 +446,7 @@ int fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, fl
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H,
                int N, int d, int causal, float scale, void* stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
-  if (B < 1 || H < 1 || N < 1 || !isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || !(scale > 0.f) || !isfinite(scale)) return FA_ERR_INVALID_ARG;
   if (d < 1 || d > 128 || (d % 4) != 0) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H > 65535 || static_cast<long double>(B) * N * H * d > 9.0e15L)
     return FA_ERR_INVALID_ARG;

@@ -57,6 +57,7 @@ struct Bars {
   uint32_t tmem_base;
   Abort abort;
 };
+static_assert(sizeof(Bars) <= 256, "barrier block larger than its shared-memory region");
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)

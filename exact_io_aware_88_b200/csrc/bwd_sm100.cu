@@ -88,6 +88,7 @@ struct Bars {
   uint32_t tmem_base;
   Abort abort;
 };
+static_assert(sizeof(Bars) <= 256, "barrier block larger than its shared-memory region");
 
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(

@@ -18,7 +18,8 @@
 //   warps 4-7   softmax for query tile 1
 //   warp  8     TMA producer (one lane);  warp 9: TMEM allocator + tcgen05.mma issuer
 //   warps 10-11 idle
-// TMEM (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+// TMEM (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,384), O1 [384,512); P_t
+// (bf16 pairs) overwrites the first half of S_t, O_t uses the first D columns of its slot.
 //
 // Tensor-core issue order per K/V tile j (after S0(0), S1(0)):
 //   PV0(j), S0(j+1), PV1(j), S1(j+1)
@@ -69,8 +70,9 @@ struct Cfg {
   static constexpr int kOffK = kOffQ + 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kSmemBytes = kOffBar + 256;    // base is 1024-aligned (checked)
-  static constexpr uint32_t kColO = 256;
+  static constexpr int kBarBytes = 512;              // Bars (size checked below)
+  static constexpr int kSmemBytes = kOffBar + kBarBytes;  // base is 1024-aligned (checked)
+  static constexpr uint32_t kColO = 256;  // O_t at kColO + 128 t
 };
 
 struct Bars {
@@ -81,6 +83,8 @@ struct Bars {
   uint32_t tmem_base;
   Abort abort;
 };
+static_assert(sizeof(Bars) <= Cfg<64>::kBarBytes && sizeof(Bars) <= Cfg<128>::kBarBytes,
+              "barrier block larger than its shared-memory region");
 
 // Unit schedule shared by every role.  Round r hands CTA c the unit r*G + c (even r) or
 // r*G + G-1-c (odd r): a snake over the persistent grid.  Under the causal mask units are
@@ -110,6 +114,24 @@ __device__ __forceinline__ Unit decode_unit(int u, int BH, int num_pairs) {
 template <bool CAUSAL>
 __device__ __forceinline__ int kv_tiles(int pair, int t, int kv_total) {
   return CAUSAL ? min(kv_total, 2 * pair + t + 1) : kv_total;
+}
+
+// Maximum of n values as a tree of 3-input max operations (depth log3 n).
+template <int n>
+__device__ __forceinline__ float tree_max(const float* v) {
+  if constexpr (n == 1) {
+    return v[0];
+  } else if constexpr (n == 2) {
+    return fmaxf(v[0], v[1]);
+  } else {
+    constexpr int m = (n + 2) / 3;
+    float w[m];
+#pragma unroll
+    for (int i = 0; i < n / 3; ++i) w[i] = max3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+    if constexpr (n % 3 == 1) w[m - 1] = v[n - 1];
+    if constexpr (n % 3 == 2) w[m - 1] = fmaxf(v[n - 2], v[n - 1]);
+    return tree_max<m>(w);
+  }
 }
 
 template <int D, bool CAUSAL>
@@ -173,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = (warp & 3) * 32 + lane;  // row within the tile == TMEM lane
     const uint32_t lane_base = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t colS = BN * t;
-    const uint32_t colO = C::kColO + D * t;
+    const uint32_t colO = C::kColO + 128 * t;
     int ns = 0;     // s_full phases consumed
     int units = 0;  // units finished
     bool ok = true;
@@ -214,13 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < BN; ++i)
             if (i > lim) sv[i] = -INFINITY;
         }
-        float mx;
-        {
-          float m4[4] = {sv[0], sv[1], sv[2], sv[3]};  // 4 independent chains
-#pragma unroll
-          for (int i = 4; i < BN; i += 2) m4[(i >> 1) & 3] = max3(m4[(i >> 1) & 3], sv[i], sv[i + 1]);
-          mx = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
-        }
+        const float mx = tree_max<BN>(sv);
         const float m_tile = mx * scale_log2;
         float alpha = 1.f;
         bool need = false;
@@ -231,26 +247,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = m_tile;
           need = true;
         }
-        // p = exp2(s * scale*log2(e) - m).  On unmasked tiles a fixed share of the pairs
-        // uses the FMA-pipe exp2 (packed fp32 pairs) so the MUFU unit and the FMA pipe share
-        // the exponentials; masked tiles use the hardware exp2 only, which maps the masked
-        // -inf logits to exact zeros.
+        // p = exp2(s * scale*log2(e) - m), two elements per packed FFMA.  On unmasked tiles
+        // a fixed share of the pairs uses the FMA-pipe exp2 so that the MUFU unit and the
+        // FMA pipe share the exponentials; masked tiles use the hardware exp2 only, which
+        // maps the masked -inf logits to exact zeros.
         const uint64_t c2 = f2_pack(scale_log2, scale_log2);
         const uint64_t nm2 = f2_pack(-m, -m);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        uint64_t acc2[2] = {0ull, 0ull};
         uint32_t pk[BN / 2];
         auto softmax_pairs = [&](auto emulate) {
 #pragma unroll
           for (int i = 0; i < BN / 2; ++i) {
-            float p0, p1;
+            const uint64_t xs = f2_fma(f2_pack(sv[2 * i], sv[2 * i + 1]), c2, nm2);
+            uint64_t p2;
             if (decltype(emulate)::value && (i % 8) < kEmuPairsPer8<D>) {
-              f2_unpack(exp2_poly2(f2_fma(f2_pack(sv[2 * i], sv[2 * i + 1]), c2, nm2)), p0, p1);
+              p2 = exp2_poly2(xs);
             } else {
-              p0 = ex2_approx(fmaf(sv[2 * i], scale_log2, -m));
-              p1 = ex2_approx(fmaf(sv[2 * i + 1], scale_log2, -m));
+              float x0, x1;
+              f2_unpack(xs, x0, x1);
+              p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
             }
-            acc[(2 * i) & 3] += p0;
-            acc[(2 * i + 1) & 3] += p1;
+            acc2[i & 1] = f2_add(acc2[i & 1], p2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
             pk[i] = pack_bf16x2(p0, p1);
           }
         };
@@ -259,8 +278,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           softmax_pairs(std::true_type{});
         }
-        const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        l = l * alpha + sum;
+        {
+          float s0, s1, s2, s3;
+          f2_unpack(acc2[0], s0, s1);
+          f2_unpack(acc2[1], s2, s3);
+          l = l * alpha + ((s0 + s1) + (s2 + s3));
+        }
         // P (bf16 pairs) into the first 64 columns of this tile's S region.
         tmem_st32(lane_base + colS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
         tmem_st32(lane_base + colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
@@ -391,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t vb = aV + s * C::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
-            umma_ts(tbase + C::kColO + D * t, tbase + BN * t + kk * 8,
+            umma_ts(tbase + C::kColO + 128 * t, tbase + BN * t + kk * 8,
                     sdesc_sw128(vb + kk * 2048, C::kChunkBytes, 1024), idesc_o,
                     (!first || kk > 0) ? 1u : 0u);
         };

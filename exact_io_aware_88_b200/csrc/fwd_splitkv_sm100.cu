@@ -62,6 +62,8 @@ struct Bars {
   uint32_t tmem_base;
   Abort abort;
 };
+// The block-sparse tile count sits at byte 248 of the 256-byte barrier region.
+static_assert(sizeof(Bars) <= 248, "barrier block larger than its shared-memory region");
 
 template <bool F16>
 __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {

@@ -18,7 +18,8 @@
  *  - lse[b][h][i] = ln sum_j exp(scale * q_i . k_j) over the keys visible to query i
  *    (natural log, scale included).
  *  - Causal mask: key j is visible to query i iff j <= i.  Q and K have the same length N.
- *  - scale is passed explicitly (1/sqrt(d) gives the textbook softmax).
+ *  - scale is passed explicitly (1/sqrt(d) gives the textbook softmax); it must be a
+ *    positive finite number (the kernels take each row maximum before scaling).
  *  - All tensor pointers are DEVICE pointers owned by the caller.  No entry point
  *    allocates, frees or synchronises (except fa_read_device_status); work is enqueued on
  *    `stream` (a cudaStream_t passed as void*, NULL = legacy default stream).
@@ -42,7 +43,7 @@ extern "C" {
 
 typedef enum {
   FA_OK = 0,
-  FA_ERR_INVALID_ARG = 1, /* B, H or N < 1, a null pointer, non-finite scale, size overflow */
+  FA_ERR_INVALID_ARG = 1, /* B, H or N < 1, a null pointer, scale not > 0 and finite, size overflow */
   FA_ERR_UNSUPPORTED = 2, /* head dim not supported by this entry point / no sm_100 device */
   FA_ERR_MISALIGNED = 3,  /* a pointer not 16-byte aligned                                */
   FA_ERR_WORKSPACE = 4,   /* workspace null or smaller than fa_bwd_workspace_bytes()      */

@@ -62,6 +62,8 @@ A16 = 1 << 20  # a fake, 16-byte aligned "device address": never dereferenced
     (dict(N=-1), 1),
     (dict(scale=float("nan")), 1),
     (dict(scale=float("inf")), 1),
+    (dict(scale=0.0), 1),
+    (dict(scale=-0.125), 1),
     (dict(d=96), 2),
     (dict(d=256), 2),
     (dict(q=A16 + 8), 3),
