@@ -9,3 +9,4 @@ from .attention import (  # noqa: F401
     forward, backward, forward_head, backward_head,
     forward_rows, dq_rows, kv_grad_tail, scalar_loop_head, forward_head_block_sparse,
 )
+from . import fp8  # noqa: F401,E402

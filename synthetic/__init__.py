@@ -141,3 +141,40 @@ def decode_workloads():
         for Nk in (4096, 16384, 65536):
             out.append((f"decode_q{Nq}_k{Nk}", 8, Nq, Nk, 16, 128, 1005))
     return out
+
+
+def draw_outliers(B: int, N: int, H: int, d: int, seed: int, frac: float = 1e-3,
+                  mag: float = 10.0) -> Dict[str, torch.Tensor]:
+    """q, k, v [B, N, H, d] bf16 with rare large entries, for the FP8 error study: every entry
+    is a standard normal, and an entry chosen with probability `frac` is multiplied by
+    `mag`.  Drawn in the order q, k, v; for each tensor the normals first, then the uniforms
+    that pick the outliers."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    out = {}
+    for nm in ("q", "k", "v"):
+        t = torch.randn((B, N, H, d), generator=g, dtype=torch.float32)
+        u = torch.rand((B, N, H, d), generator=g, dtype=torch.float32)
+        t = torch.where(u < frac, t * mag, t)
+        out[nm] = t.to(torch.bfloat16).contiguous()
+    return out
+
+
+def draw_signs(d: int, seed: int) -> torch.Tensor:
+    """The random +-1 diagonal of the incoherent-processing transform, fp32 [d]."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    bits = torch.randint(0, 2, (d,), generator=g, dtype=torch.int64)
+    return (1.0 - 2.0 * bits.to(torch.float32)).contiguous()
+
+
+def fp8_workloads():
+    """FP8 forward shapes: the head-dim-128 rows of the prefill sweep at 4k and 16k tokens
+    per sequence, causal and not (B*N = 16384, H = 16).  Returns (name, B, N, H, d, causal,
+    seed)."""
+    out = []
+    for N in (4096, 16384):
+        for causal in (False, True):
+            nm = f"fwd_fp8:B{TOTAL_TOKENS // N}xN{N}xH16xd128" + ("-causal" if causal else "")
+            out.append((nm, TOTAL_TOKENS // N, N, 16, 128, causal, 1006))
+    return out
