@@ -492,6 +492,41 @@ def run_sweep(path: str, reps: int = 20, warmup: int = 3):
             print(json.dumps(rec), file=sys.stderr)
             del q, k, v, o, lse, ws, t
             torch.cuda.empty_cache()
+        # FP8 forward (E4M3 products, Hadamard-transformed Q and K): tensor-bound against the
+        # bf16 measured peak x 2 (the nominal fp8 / bf16 ratio); the operand preparation
+        # (fa_fp8_quantize) is timed separately and is HBM-bound.
+        for name, B, N, H, d, causal, seed in synthetic.fp8_workloads():
+            t = synthetic.draw(B, N, H, d, seed, "bf16")
+            q, k, v = (t[n].to(dev) for n in ("q", "k", "v"))
+            signs = synthetic.draw_signs(d, seed + 1).to(dev)
+            npad = (N + 15) // 16 * 16
+            q8 = torch.empty((B, N, H, d), device=dev, dtype=torch.uint8)
+            k8 = torch.empty_like(q8)
+            vt8 = torch.empty((B, H, d, npad), device=dev, dtype=torch.uint8)
+            sc = torch.empty((3, B * H), device=dev, dtype=torch.float32)
+            nb = fa.fa_fp8_quantize_workspace_bytes(B, H)
+            ws = torch.empty(nb, device=dev, dtype=torch.uint8)
+            quant = lambda: fa.fa_fp8_quantize(q, k, v, signs, q8, k8, vt8, sc, B, H, N, d, ws, nb,
+                                               stream)
+            assert quant() == 0
+            qmed, qbest = timed(quant)
+            o = torch.empty_like(q)
+            lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+            f8 = lambda: fa.fa_fwd_fp8(q8, k8, vt8, sc, o, lse, B, H, N, d, causal,
+                                       1.0 / math.sqrt(d), stream)
+            assert f8() == 0
+            med, best = timed(f8)
+            flops = 4.0 * B * H * N * N * d * (0.5 if causal else 1.0)
+            rec = {"workload": name + "-e4m3", "pass": "fwd_fp8", "ms": round(med, 4),
+                   "ms_best": round(best, 4), "tflops": round(flops / (med * 1e-3) / 1e12, 1),
+                   "frac_of_fp8_peak": round(flops / (med * 1e-3) / 1e12 / (2 * burst), 4),
+                   "quantize_ms": round(qmed, 4),
+                   "quantize_gbs": round(3 * B * N * H * d * (2 + 2 + 1) / (qmed * 1e-3) / 1e9, 1),
+                   "peak_source": peak_src + " (fp8 peak = 2 x measured bf16 burst)"}
+            out.write(json.dumps(rec) + "\n")
+            print(json.dumps(rec), file=sys.stderr)
+            del q, k, v, q8, k8, vt8, sc, ws, o, lse, t
+            torch.cuda.empty_cache()
     if fa.fa_read_device_status(stream) != 0:
         raise RuntimeError("device status word reports a timeout")
 

@@ -81,16 +81,35 @@ int check_shape(int B, int H, int N, int d, float scale) {
 
 // 4-D view [B][N][H][d] (innermost first: d, H, N, B) of a bf16 tensor, tiled in boxes of
 // 64 d-elements (128 bytes, the 128-byte swizzle span) x 1 head x 128 rows x 1 batch.
+// 8-bit tensors (E4M3 codes as UINT8) use boxes of 128 d-elements, again 128 bytes.
 int encode_bnhd(CUtensorMap* m, const void* ptr, int B, int N, int H, int d,
                 CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+  const cuuint64_t es = (dt == CU_TENSOR_MAP_DATA_TYPE_UINT8) ? 1 : 2;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2,
-                                 static_cast<cuuint64_t>(H) * d * 2,
-                                 static_cast<cuuint64_t>(N) * H * d * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * es,
+                                 static_cast<cuuint64_t>(H) * d * es,
+                                 static_cast<cuuint64_t>(N) * H * d * es};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / es), 1, 128, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = g_encode(m, dt, 4, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// 4-D view of an 8-bit V^T [B][H][d][npad] (innermost first: keys, d, H, B), boxes of 128
+// keys (128 bytes) x 128 head-dim rows.
+int encode_vt8(CUtensorMap* m, const void* ptr, int B, int H, int d, int npad) {
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(npad), static_cast<cuuint64_t>(d),
+                              static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(npad),
+                                 static_cast<cuuint64_t>(d) * npad,
+                                 static_cast<cuuint64_t>(H) * d * npad};
+  const cuuint32_t box[4] = {128, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(ptr), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -175,6 +194,75 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   a.status = di.status;
   a.num_sms = di.num_sms;
   return from_cuda(fa::launch_fwd_sm100(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t fa_fp8_quantize_workspace_bytes(int B, int H) {
+  if (B < 1 || H < 1 || static_cast<long long>(B) * H > 0x7fffffffLL / 3) return 0;
+  return round_up(3 * sizeof(uint32_t) * static_cast<size_t>(B) * H, 256);
+}
+
+int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* signs, void* q8,
+                    void* k8, void* vt8, float* scales, int B, int H, int N, int d,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !q8 || !k8 || !vt8 || !scales) return FA_ERR_INVALID_ARG;
+  int rc = check_shape(B, H, N, d, 1.0f);
+  if (rc) return rc;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(q8, 16) ||
+      !aligned(k8, 16) || !aligned(vt8, 16) || !aligned(scales, 4) ||
+      (signs && !aligned(signs, 4)))
+    return FA_ERR_MISALIGNED;
+  const size_t need = fa_fp8_quantize_workspace_bytes(B, H);
+  if (!workspace || need == 0 || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned(workspace, 4)) return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  fa::Fp8QuantArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.signs = signs;
+  a.q8 = q8;
+  a.k8 = k8;
+  a.vt8 = vt8;
+  a.scales = scales;
+  a.amax = static_cast<uint32_t*>(workspace);
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.d = d;
+  return from_cuda(fa::launch_fp8_quantize(a, static_cast<cudaStream_t>(stream)));
+}
+
+int fa_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* scales, void* o,
+               float* lse, int B, int H, int N, int d, int causal, float scale, void* stream) {
+  if (!q8 || !k8 || !vt8 || !scales || !o || !lse) return FA_ERR_INVALID_ARG;
+  int rc = check_shape(B, H, N, d, scale);
+  if (rc) return rc;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(vt8, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || !aligned(scales, 4))
+    return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  fa::FwdArgs a;
+  const int npad = (N + 15) / 16 * 16;
+  if ((rc = encode_bnhd(&a.tm_q, q8, B, N, H, d, CU_TENSOR_MAP_DATA_TYPE_UINT8)) ||
+      (rc = encode_bnhd(&a.tm_k, k8, B, N, H, d, CU_TENSOR_MAP_DATA_TYPE_UINT8)) ||
+      (rc = encode_vt8(&a.tm_v, vt8, B, H, d, npad)))
+    return rc;
+  a.o = o;
+  a.lse = lse;
+  a.scales = scales;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.d = d;
+  a.causal = causal ? 1 : 0;
+  a.scale = scale;
+  a.status = di.status;
+  a.num_sms = di.num_sms;
+  return from_cuda(fa::launch_fwd_fp8(a, static_cast<cudaStream_t>(stream)));
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {

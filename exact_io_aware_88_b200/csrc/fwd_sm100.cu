@@ -57,15 +57,20 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Pairs out of every 8 whose exp2 runs on the FMA pipe (exp2_poly2) instead of the MUFU
 // unit, on unmasked tiles.  Measured on B200: with head dim 64 (half the tensor work per
 // tile) moving 2 of 8 pairs is best (+4 %; 4 of 8 is slower); head dim 128 gains nothing.
-template <int D>
-constexpr int kEmuPairsPer8 = (D == 64) ? 2 : 0;
+// The 8-bit path has the same tensor time per tile as head dim 64 in bf16.
+template <int D, bool F8>
+constexpr int kEmuPairsPer8 = (D == 64 || F8) ? 2 : 0;
 
-template <int D>
+// F8: Q, K and V^T are E4M3 (one byte per element); otherwise bf16.
+template <int D, bool F8 = false>
 struct Cfg {
-  static constexpr int kChunks = D / 64;              // 64-element (128-byte) column chunks
+  static constexpr int kElem = F8 ? 1 : 2;
+  static constexpr int kRowBytes = D * kElem;         // one head-dim row of Q or K
+  static constexpr int kChunks = kRowBytes / 128;     // 128-byte column chunks
+  static constexpr int kChunkElems = 128 / kElem;
   static constexpr int kChunkBytes = BM * 128;        // one TMA box: 128 rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStages = (D == 128) ? 2 : 4;  // K/V ring depth
+  static constexpr int kStages = (kChunks == 2) ? 2 : 4;  // K/V ring depth
   static constexpr int kOffQ = 0;                     // Q0, Q1
   static constexpr int kOffK = kOffQ + 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
@@ -134,13 +139,15 @@ __device__ __forceinline__ float tree_max(const float* v) {
   }
 }
 
-template <int D, bool CAUSAL>
+// F8: tm_q / tm_k map E4M3 [B][N][H][d], tm_v maps E4M3 V^T [B][H][d][Npad] (keys
+// contiguous), and scales[3][B*H] holds the per-head dequantisation scales of Q, K, V.
+template <int D, bool CAUSAL, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
-               float* __restrict__ lse, int B, int H, int N, float scale_log2, int num_pairs,
-               int* status, uint64_t timeout_ns) {
-  using C = Cfg<D>;
+               float* __restrict__ lse, const float* __restrict__ scales, int B, int H, int N,
+               float scale_log2, int num_pairs, int* status, uint64_t timeout_ns) {
+  using C = Cfg<D, F8>;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {  // 128-byte-swizzled tiles need a 1024-aligned base
     if (threadIdx.x == 0) atomicCAS(status, FA_OK, FA_ERR_UNSUPPORTED);
@@ -207,6 +214,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int q0 = (2 * x.pair + t) * BM;
       const int row = q0 + r;
       const int nkv = kv_tiles<CAUSAL>(x.pair, t, kv_total);
+      // Logit scale in log2 units (8-bit path: times the Q and K dequantisation scales) and
+      // the output's extra factor (8-bit path: V's scale).
+      float sl2 = scale_log2, out_mul = 1.f;
+      if constexpr (F8) {
+        sl2 *= scales[x.bh] * scales[BH + x.bh];
+        out_mul = scales[2 * BH + x.bh];
+      }
       float m = -INFINITY;  // running max of scale*log2(e)*s (possibly stale by < 2^8)
       float l = 0.f;
       for (int j = 0; j < nkv; ++j) {
@@ -237,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (i > lim) sv[i] = -INFINITY;
         }
         const float mx = tree_max<BN>(sv);
-        const float m_tile = mx * scale_log2;
+        const float m_tile = mx * sl2;
         float alpha = 1.f;
         bool need = false;
         if (m == -INFINITY) {
@@ -251,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // a fixed share of the pairs uses the FMA-pipe exp2 so that the MUFU unit and the
         // FMA pipe share the exponentials; masked tiles use the hardware exp2 only, which
         // maps the masked -inf logits to exact zeros.
-        const uint64_t c2 = f2_pack(scale_log2, scale_log2);
+        const uint64_t c2 = f2_pack(sl2, sl2);
         const uint64_t nm2 = f2_pack(-m, -m);
         uint64_t acc2[2] = {0ull, 0ull};
         uint32_t pk[BN / 2];
@@ -260,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < BN / 2; ++i) {
             const uint64_t xs = f2_fma(f2_pack(sv[2 * i], sv[2 * i + 1]), c2, nm2);
             uint64_t p2;
-            if (decltype(emulate)::value && (i % 8) < kEmuPairsPer8<D>) {
+            if (decltype(emulate)::value && (i % 8) < kEmuPairsPer8<D, F8>) {
               p2 = exp2_poly2(xs);
             } else {
               float x0, x1;
@@ -270,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc2[i & 1] = f2_add(acc2[i & 1], p2);
             float p0, p1;
             f2_unpack(p2, p0, p1);
-            pk[i] = pack_bf16x2(p0, p1);
+            pk[i] = F8 ? pack_e4m3x2(p0, p1) : pack_bf16x2(p0, p1);
           }
         };
         if (masked) {
@@ -284,9 +298,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           f2_unpack(acc2[1], s2, s3);
           l = l * alpha + ((s0 + s1) + (s2 + s3));
         }
-        // P (bf16 pairs) into the first 64 columns of this tile's S region.
-        tmem_st32(lane_base + colS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(lane_base + colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        // P into the first columns of this tile's S region: bf16 pairs (64 columns) or
+        // E4M3 quads (32 columns).
+        if constexpr (F8) {
+          uint32_t w[BN / 4];
+#pragma unroll
+          for (int i = 0; i < BN / 4; ++i) w[i] = pk[2 * i] | (pk[2 * i + 1] << 16);
+          tmem_st32(lane_base + colS, w);
+        } else {
+          tmem_st32(lane_base + colS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+          tmem_st32(lane_base + colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        }
         if (__any_sync(0xffffffffu, need)) {
           // O_t holds sum_{j'<j} P V, and PV_t(j-1) has completed: it precedes S_t(j).
 #pragma unroll
@@ -315,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bars->o_free[t]);  // the next unit's first PV may overwrite O_t now
       ++units;
       if (row < N) {
-        const float inv_l = 1.f / l;
+        const float inv_l = out_mul / l;
         __nv_bfloat16* orow = out + ((static_cast<size_t>(b) * N + row) * H + h) * D;
 #pragma unroll
         for (int c8 = 0; c8 < D / 8; ++c8)
@@ -352,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t < 2; ++t)
             for (int c = 0; c < C::kChunks; ++c)
               tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &tm_q, &bars->q_full,
-                          c * 64, h, (2 * x.pair + t) * BM, b, pol_q);
+                          c * C::kChunkElems, h, (2 * x.pair + t) * BM, b, pol_q);
           ++units;
           const int nkv = kv_tiles<CAUSAL>(x.pair, 1, kv_total);
           for (int j = 0; j < nkv; ++j, ++g) {
@@ -364,16 +386,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes);
             for (int c = 0; c < C::kChunks; ++c)
               tma_load_4d(sK + s * C::kTileBytes + c * C::kChunkBytes, &tm_k, &bars->k_full[s],
-                          c * 64, h, j * BN, b, pol_kv);
+                          c * C::kChunkElems, h, j * BN, b, pol_kv);
             if (g >= C::kStages &&
                 !(ok = mbar_wait(&bars->v_empty[s], ph, ab, status, timeout_ns))) {
               ++g;  // K of this tile is in flight: count it for the drain below
               break;
             }
             mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
-            for (int c = 0; c < C::kChunks; ++c)
-              tma_load_4d(sV + s * C::kTileBytes + c * C::kChunkBytes, &tm_v, &bars->v_full[s],
-                          c * 64, h, j * BN, b, pol_kv);
+            if constexpr (F8) {  // V^T box: 128 keys x 128 head-dim rows
+              tma_load_4d(sV + s * C::kTileBytes, &tm_v, &bars->v_full[s], j * BN, 0, h, b,
+                          pol_kv);
+            } else {
+              for (int c = 0; c < C::kChunks; ++c)
+                tma_load_4d(sV + s * C::kTileBytes + c * C::kChunkBytes, &tm_v, &bars->v_full[s],
+                            c * 64, h, j * BN, b, pol_kv);
+            }
           }
         }
         // Drain: no copy into shared memory may still be in flight when the CTA exits.
@@ -392,8 +419,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kWarpMma) {
       // ---------------------------------------------------------------- MMA issuer
       if (lane == 0) {
-        constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
-        constexpr uint32_t idesc_o = idesc_bf16_f32(BM, D, 0, 1);
+        constexpr uint32_t idesc_s = F8 ? idesc_e4m3_f32(BM, BN, 0, 0) : idesc_bf16_f32(BM, BN, 0, 0);
+        // PV: bf16 V is [keys][d] (MN-major B); the 8-bit V^T is [d][keys] (K-major B).
+        constexpr uint32_t idesc_o = F8 ? idesc_e4m3_f32(BM, D, 0, 0) : idesc_bf16_f32(BM, D, 0, 1);
         const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
         int g = 0;            // K/V tiles consumed so far (ring position)
         int units = 0;        // units finished
@@ -402,21 +430,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto issue_s = [&](int t, int s) {  // S_t = Q_t K^T (both K-major over the head dim)
           const uint32_t kb = aK + s * C::kTileBytes;
           const uint32_t qb = aQ + t * C::kTileBytes;
+          // One MMA per 32 bytes of the head dim (16 bf16 or 32 E4M3 elements).
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
+          for (int kk = 0; kk < C::kRowBytes / 32; ++kk) {
             const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-            umma_ss(tbase + BN * t, sdesc_sw128(qb + off, 16, 1024),
-                    sdesc_sw128(kb + off, 16, 1024), idesc_s, kk > 0);
+            if constexpr (F8)
+              umma_ss_f8(tbase + BN * t, sdesc_sw128(qb + off, 16, 1024),
+                         sdesc_sw128(kb + off, 16, 1024), idesc_s, kk > 0);
+            else
+              umma_ss(tbase + BN * t, sdesc_sw128(qb + off, 16, 1024),
+                      sdesc_sw128(kb + off, 16, 1024), idesc_s, kk > 0);
           }
           umma_commit(&bars->s_full[t]);
         };
         auto issue_pv = [&](int t, int s, bool first) {  // O_t += P_t V (P from TMEM)
           const uint32_t vb = aV + s * C::kTileBytes;
+          if constexpr (F8) {  // 32 keys per MMA: 8 TMEM columns of P, 32 bytes of V^T rows
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            umma_ts(tbase + C::kColO + 128 * t, tbase + BN * t + kk * 8,
-                    sdesc_sw128(vb + kk * 2048, C::kChunkBytes, 1024), idesc_o,
-                    (!first || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BN / 32; ++kk)
+              umma_ts_f8(tbase + C::kColO + 128 * t, tbase + BN * t + kk * 8,
+                         sdesc_sw128(vb + kk * 32, 16, 1024), idesc_o, (!first || kk > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk)
+              umma_ts(tbase + C::kColO + 128 * t, tbase + BN * t + kk * 8,
+                      sdesc_sw128(vb + kk * 2048, C::kChunkBytes, 1024), idesc_o,
+                      (!first || kk > 0) ? 1u : 0u);
+          }
         };
         for (int r = 0; ok; ++r) {
           const int u = unit_of_round(r, G);
@@ -496,10 +536,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool F8 = false>
 static cudaError_t launch_t(const FwdArgs& a, cudaStream_t st) {
-  using C = Cfg<D>;
-  auto kern = fwd_kernel<D, CAUSAL>;
+  using C = Cfg<D, F8>;
+  auto kern = fwd_kernel<D, CAUSAL, F8>;
   // The setmaxnreg split assumes the kernel launches with exactly kRegsLaunch registers per
   // thread; with fewer, the softmax warpgroups' increase could never be satisfied.
   cudaFuncAttributes fa_attr;
@@ -514,8 +554,8 @@ static cudaError_t launch_t(const FwdArgs& a, cudaStream_t st) {
   const int grid = static_cast<int>(std::min<long long>(units, a.num_sms));
   const float scale_log2 = a.scale * 1.4426950408889634f;
   kern<<<grid, kThreads, C::kSmemBytes, st>>>(a.tm_q, a.tm_k, a.tm_v,
-                                              static_cast<__nv_bfloat16*>(a.o), a.lse, a.B, a.H,
-                                              a.N, scale_log2, num_pairs, a.status,
+                                              static_cast<__nv_bfloat16*>(a.o), a.lse, a.scales,
+                                              a.B, a.H, a.N, scale_log2, num_pairs, a.status,
                                               kDefaultWaitTimeoutNs);
   return cudaGetLastError();
 }
@@ -525,6 +565,11 @@ static cudaError_t launch_t(const FwdArgs& a, cudaStream_t st) {
 cudaError_t launch_fwd_sm100(const FwdArgs& a, cudaStream_t s) {
   if (a.d == 64) return a.causal ? fwd::launch_t<64, true>(a, s) : fwd::launch_t<64, false>(a, s);
   return a.causal ? fwd::launch_t<128, true>(a, s) : fwd::launch_t<128, false>(a, s);
+}
+
+cudaError_t launch_fwd_fp8(const FwdArgs& a, cudaStream_t s) {
+  if (a.d != 128) return cudaErrorNotSupported;
+  return a.causal ? fwd::launch_t<128, true, true>(a, s) : fwd::launch_t<128, false, true>(a, s);
 }
 
 }  // namespace fa

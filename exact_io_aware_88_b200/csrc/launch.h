@@ -14,8 +14,11 @@ constexpr uint64_t kDefaultWaitTimeoutNs = 4000000000ull;
 
 struct FwdArgs {
   CUtensorMap tm_q, tm_k, tm_v;  // 4-D maps over [B][N][H][d] bf16, box {64,1,128,1}
+                                 // (8-bit path: E4M3 box {128,1,128,1}; tm_v over V^T
+                                 // [B][H][d][Npad], box {128,128,1,1})
   void* o;
   float* lse;
+  const float* scales = nullptr;  // 8-bit path: [3][B*H] dequantisation scales
   int B, H, N, d, causal;
   float scale;
   int* status;
@@ -51,6 +54,18 @@ struct SplitKvArgs {
 };
 
 cudaError_t launch_fwd_sm100(const FwdArgs& a, cudaStream_t s);
+cudaError_t launch_fwd_fp8(const FwdArgs& a, cudaStream_t s);
+
+struct Fp8QuantArgs {
+  const void *q, *k, *v;  // [B][N][H][d] bf16
+  const float* signs;     // [d] +-1, or null (no transform)
+  void *q8, *k8;          // [B][N][H][d] E4M3
+  void* vt8;              // [B][H][d][Npad] E4M3, Npad = N rounded up to 16
+  float* scales;          // [3][B*H]
+  uint32_t* amax;         // [3][B*H] workspace
+  int B, H, N, d;
+};
+cudaError_t launch_fp8_quantize(const Fp8QuantArgs& a, cudaStream_t s);
 cudaError_t launch_fwd_splitkv(const SplitKvArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_pre(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t s, bool with_dq);

@@ -75,6 +75,12 @@ _lib.fa_fwd_block_sparse_workspace_bytes.argtypes = [_I, _I, _I, _I]
 _lib.fa_fwd_block_sparse_workspace_bytes.restype = _SZ
 _lib.fa_fwd_block_sparse.argtypes = [_P] * 5 + [_I] * 5 + [_F, _P, _P, _SZ, _P]
 _lib.fa_fwd_block_sparse.restype = _I
+_lib.fa_fp8_quantize_workspace_bytes.argtypes = [_I, _I]
+_lib.fa_fp8_quantize_workspace_bytes.restype = _SZ
+_lib.fa_fp8_quantize.argtypes = [_P] * 8 + [_I] * 4 + [_P, _SZ, _P]
+_lib.fa_fp8_quantize.restype = _I
+_lib.fa_fwd_fp8.argtypes = [_P] * 6 + [_I] * 5 + [_F, _P]
+_lib.fa_fwd_fp8.restype = _I
 _lib.fa_fwd_f32.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.fa_fwd_f32.restype = _I
 _lib.fa_read_device_status.argtypes = [ctypes.POINTER(_I), _P]
@@ -94,6 +100,7 @@ _lib.fa_debug_wait_timeout.restype = _I
 EXPORTED = sorted(["fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess", "fa_bwd_kv",
                    "fa_bwd_dq_convert", "fa_bwd_noalloc", "fa_fwd_f32", "fa_fwd_splitkv",
                    "fa_fwd_splitkv_workspace_bytes", "fa_fwd_block_sparse",
+                   "fa_fp8_quantize_workspace_bytes", "fa_fp8_quantize", "fa_fwd_fp8",
                    "fa_fwd_block_sparse_workspace_bytes", "fa_read_device_status", "fa_status_string",
                    "fa_version", "fa_debug_umma_tile", "fa_debug_wait_timeout",
                    "fa_debug_exp2"])
@@ -186,6 +193,22 @@ def fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, dtype, works
     return _lib.fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
                                int(causal), float(scale), int(dtype), _ptr(workspace),
                                int(workspace_bytes), _stream(stream))
+
+
+def fa_fp8_quantize_workspace_bytes(B, H) -> int:
+    return _lib.fa_fp8_quantize_workspace_bytes(B, H)
+
+
+def fa_fp8_quantize(q, k, v, signs, q8, k8, vt8, scales, B, H, N, d, workspace, workspace_bytes,
+                    stream=None) -> int:
+    return _lib.fa_fp8_quantize(_ptr(q), _ptr(k), _ptr(v), _ptr(signs), _ptr(q8), _ptr(k8),
+                                _ptr(vt8), _ptr(scales), B, H, N, d, _ptr(workspace),
+                                int(workspace_bytes), _stream(stream))
+
+
+def fa_fwd_fp8(q8, k8, vt8, scales, o, lse, B, H, N, d, causal, scale, stream=None) -> int:
+    return _lib.fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(vt8), _ptr(scales), _ptr(o), _ptr(lse), B, H,
+                           N, d, int(causal), float(scale), _stream(stream))
 
 
 def fa_fwd_block_sparse_workspace_bytes(B, H, N, d) -> int:
@@ -299,4 +322,35 @@ def attention_block_sparse(q, k, v, block_mask: torch.Tensor, causal: bool = Fal
     ws = torch.empty(max(nb, 256), device=q.device, dtype=torch.uint8)
     _check("fa_fwd_block_sparse", fa_fwd_block_sparse(q, k, v, o, lse, B, H, N, d, causal, scale,
                                                       m, ws, ws.numel()))
+    return o, lse
+
+
+def fp8_quantize(q, k, v, signs: Optional[torch.Tensor]):
+    """E4M3 operands for attention_forward_fp8 from bf16 [B, N, H, d] q, k, v; signs is the
+    [d] +-1 diagonal of the Hadamard transform (None: no transform).  Returns
+    (q8, k8, vt8, scales) as uint8 [B, N, H, d], uint8 [B, N, H, d], uint8 [B, H, d, Npad]
+    and fp32 [3, B*H]."""
+    B, N, H, d = _shape(q)
+    npad = (N + 15) // 16 * 16
+    dev = q.device
+    q8 = torch.empty((B, N, H, d), device=dev, dtype=torch.uint8)
+    k8 = torch.empty_like(q8)
+    vt8 = torch.empty((B, H, d, npad), device=dev, dtype=torch.uint8)
+    scales = torch.empty((3, B * H), device=dev, dtype=torch.float32)
+    nb = fa_fp8_quantize_workspace_bytes(B, H)
+    ws = torch.empty(max(nb, 256), device=dev, dtype=torch.uint8)
+    sg = None if signs is None else signs.to(device=dev, dtype=torch.float32).contiguous()
+    _check("fa_fp8_quantize", fa_fp8_quantize(q, k, v, sg, q8, k8, vt8, scales, B, H, N, d, ws,
+                                              ws.numel()))
+    return q8, k8, vt8, scales
+
+
+def attention_forward_fp8(q8, k8, vt8, scales, causal: bool = False,
+                          scale: Optional[float] = None):
+    """O (bf16 [B, N, H, d]) and LSE (fp32 [B, H, N]) from fp8_quantize's operands."""
+    B, N, H, d = q8.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty((B, N, H, d), device=q8.device, dtype=torch.bfloat16)
+    lse = torch.empty((B, H, N), device=q8.device, dtype=torch.float32)
+    _check("fa_fwd_fp8", fa_fwd_fp8(q8, k8, vt8, scales, o, lse, B, H, N, d, causal, scale))
     return o, lse

@@ -166,6 +166,39 @@ int fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, fl
                         const uint8_t* block_mask, void* workspace, size_t workspace_bytes,
                         void* stream);
 
+/* FP8 forward with incoherent processing ("FlashAttention-3 — FlashAttention-3", section
+ * FlashAttention-3の技術的革新, item 3: Q and K are multiplied by a random orthogonal
+ * matrix -- a Hadamard matrix -- before the 8-bit rounding; the matrix cancels in Q K^T).
+ * Two calls: fa_fp8_quantize prepares the operands once, fa_fwd_fp8 runs attention on them
+ * with both products on the tensor core in E4M3 (kind::f8f6f4).
+ *
+ * fa_fp8_quantize:
+ *   q, k, v : [B][N][H][d] bf16 (d in {64, 128}).
+ *   signs   : DEVICE [d] fp32 of +-1 (the random diagonal s), or NULL for no transform.
+ *             Q and K rows are mapped x -> x diag(s) H_d / sqrt(d), H_d the Sylvester
+ *             Hadamard matrix of order d.
+ *   q8, k8  : [B][N][H][d] E4M3 codes (1 byte each); vt8 : [B][H][d][Npad] E4M3 codes of V
+ *             transposed (keys contiguous), Npad = N rounded up to a multiple of 16, keys
+ *             in [N, Npad) zero.  No transform on V.
+ *   scales  : [3][B*H] fp32, the dequantisation scales of Q, K, V per (batch, head): the
+ *             smallest power of two 2^e with 448 * 2^e >= max |x| over the (transformed)
+ *             head (1 for an all-zero head); codes are round-to-nearest-even, saturating
+ *             E4M3 of x / 2^e.
+ *   workspace : >= fa_fp8_quantize_workspace_bytes(B, H) bytes, 4-byte aligned (per-head
+ *             maxima; cleared by the call).
+ * fa_fwd_fp8:
+ *   q8, k8, vt8, scales : as produced above, d = 128 only (others: FA_ERR_UNSUPPORTED).
+ *   o : [B][N][H][d] bf16, lse : [B][H][N] fp32, for
+ *       O = softmax(scale * (s_q Q8)(s_k K8)^T) (s_v V8) with P rounded to E4M3 before the
+ *       second product; lse is that softmax's natural-log normaliser.
+ *   Errors as fa_fwd; all pointers DEVICE, 16-byte aligned (scales, lse: 4). */
+size_t fa_fp8_quantize_workspace_bytes(int B, int H);
+int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* signs,
+                    void* q8, void* k8, void* vt8, float* scales, int B, int H, int N, int d,
+                    void* workspace, size_t workspace_bytes, void* stream);
+int fa_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* scales, void* o,
+               float* lse, int B, int H, int N, int d, int causal, float scale, void* stream);
+
 /* Forward pass in fp32 on the CUDA cores (no tensor cores, no TF32), for fp32 inputs.
  *   q, k, v, o : [B][N][H][d] fp32; lse : [B][H][N] fp32.  1 <= d <= 128, d % 4 == 0. */
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,

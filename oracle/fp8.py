@@ -25,6 +25,11 @@ Readings where the pages are silent (each one is also listed with the design not
     division by the scale exact.
   * Q and K are transformed then quantised; V is quantised without a transform (it does
     not meet K's transform in P V).
+  * The codes are decided in fp32, the kernel's precision: the transform is evaluated as
+    the textbook fast Walsh-Hadamard transform in fp32 (sign flips, then butterfly stages
+    (a + b, a - b) on pairs 1, 2, 4, ... apart, then one multiply by the fp32 value of
+    1/sqrt(d)).  ``transform`` below is the exact fp64 definition; ``transform_f32`` is
+    pinned to it within fp32 rounding.
   * The attention itself: softmax(scale * (s_q Q8)(s_k K8)^T)(s_v V8) in exact arithmetic is
     what the FP8 kernel approximates; its own further rounding (P to E4M3 for the second
     product) is an implementation error measured against this, not a reading.
@@ -59,6 +64,24 @@ def transform(X: np.ndarray, signs: Optional[np.ndarray]) -> np.ndarray:
     d = X.shape[-1]
     M = np.asarray(signs, dtype=np.float64)[:, None] * hadamard(d) / math.sqrt(d)
     return np.asarray(X, dtype=np.float64) @ M
+
+
+def transform_f32(X: np.ndarray, signs: Optional[np.ndarray]) -> np.ndarray:
+    """The transform as evaluated in fp32: x * s, log2(d) butterfly stages, times fp32
+    1/sqrt(d).  Returns fp32.  signs=None: the identity (values cast to fp32)."""
+    x = np.asarray(X, dtype=np.float32)
+    if signs is None:
+        return x
+    d = x.shape[-1]
+    x = x * np.asarray(signs, dtype=np.float32)
+    h = 1
+    while h < d:
+        y = x.reshape(*x.shape[:-1], d // (2 * h), 2, h)
+        a, b = y[..., 0, :], y[..., 1, :]
+        x = np.stack([a + b, a - b], axis=-2).reshape(*x.shape[:-1], d)
+        h *= 2
+    inv = np.float32(1.0) / np.sqrt(np.float32(d))
+    return x * inv
 
 
 def e4m3_round(x: np.ndarray) -> np.ndarray:
@@ -105,7 +128,8 @@ def e4m3_decode(codes: np.ndarray) -> np.ndarray:
 
 
 def pow2_scale(amax: float) -> float:
-    """Smallest power of two 2^e with 448 * 2^e >= amax (1.0 when amax is 0)."""
+    """Smallest power of two 2^e with 448 * 2^e >= amax (1.0 when amax is 0), e clamped
+    to [-126, 127] so that the scale is a normal fp32 number."""
     if not amax > 0:
         return 1.0
     e = math.ceil(math.log2(amax / E4M3_MAX))
@@ -113,13 +137,14 @@ def pow2_scale(amax: float) -> float:
         e -= 1
     while E4M3_MAX * 2.0 ** e < amax:
         e += 1
-    return 2.0 ** e
+    return 2.0 ** max(-126, min(127, e))  # kept a normal fp32 number
 
 
 def quantize_head(X: np.ndarray, signs: Optional[np.ndarray]) -> Tuple[np.ndarray, float, float]:
-    """One (batch, head) slice X [N, d]: transform, per-head power-of-two scale, E4M3 codes.
-    Returns (codes [N, d] uint8, scale, amax of the transformed values)."""
-    Xt = transform(X, signs)
+    """One (batch, head) slice X [N, d]: transform (in fp32, see the module notes),
+    per-head power-of-two scale, E4M3 codes.  Returns (codes [N, d] uint8, scale, amax of
+    the transformed values)."""
+    Xt = transform_f32(X, signs).astype(np.float64)
     amax = float(np.max(np.abs(Xt))) if Xt.size else 0.0
     sc = pow2_scale(amax)
     return e4m3_encode(Xt / sc), sc, amax

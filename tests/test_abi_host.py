@@ -97,6 +97,25 @@ def test_f32_rejects_bad_arguments_without_launching(fa):
     assert fa.fa_fwd_f32(A16 + 4, *p[1:], 1, 1, 16, 64, 0, 0.1, stream=0) == fa.FA_ERR_MISALIGNED
 
 
+def test_fp8_entry_points_reject_bad_arguments_without_launching(fa):
+    p = [A16] * 6
+    assert fa.fa_fwd_fp8(*p, 1, 2, 256, 64, 0, 0.1, stream=0) == fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_fwd_fp8(None, *p[1:], 1, 2, 256, 128, 0, 0.1, stream=0) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_fwd_fp8(*p, 1, 2, 256, 128, 0, -1.0, stream=0) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_fwd_fp8(A16 + 8, *p[1:], 1, 2, 256, 128, 0, 0.1, stream=0) == fa.FA_ERR_MISALIGNED
+    ws = fa.fa_fp8_quantize_workspace_bytes(2, 3)
+    assert ws == 256  # 3 * 2 * 3 words, rounded up
+    q = lambda **kw: fa.fa_fp8_quantize(
+        kw.get("q", A16), A16, A16, kw.get("signs", None), A16, A16, A16, A16, 2, 3, 100,
+        kw.get("d", 128), kw.get("ws", A16), kw.get("wsb", ws), stream=0)
+    assert q(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert q(q=None) == fa.FA_ERR_INVALID_ARG
+    assert q(ws=None) == fa.FA_ERR_WORKSPACE
+    assert q(wsb=ws - 1) == fa.FA_ERR_WORKSPACE
+    assert q(q=A16 + 2) == fa.FA_ERR_MISALIGNED
+    assert q(signs=A16 + 2) == fa.FA_ERR_MISALIGNED
+
+
 def test_debug_entry_points_reject_bad_arguments(fa):
     assert fa.fa_debug_umma_tile(A16, A16, A16, 96, 64, 0, stream=0) == fa.FA_ERR_UNSUPPORTED
     assert fa.fa_debug_umma_tile(A16, A16, A16, 64, 64, 3, stream=0) == fa.FA_ERR_UNSUPPORTED

@@ -94,6 +94,19 @@ def test_transform_matches_butterfly_and_preserves_qk(d):
     assert np.allclose(Xt @ fp8.transform(Y, s).T, X @ Y.T, rtol=0, atol=1e-11)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp32_transform_is_the_definition_within_fp32_rounding(d):
+    rng = np.random.default_rng(d + 1)
+    X = (rng.normal(size=(50, d)) * np.where(rng.random((50, d)) < 0.01, 10, 1)).astype(np.float32)
+    s = synthetic.to_f64(synthetic.draw_signs(d, 4))
+    ref = fp8.transform(X.astype(np.float64), s)
+    got = fp8.transform_f32(X, s)
+    assert got.dtype == np.float32
+    # log2(d) + 2 roundings of |values| <= sqrt(d) max|x|
+    assert np.max(np.abs(got - ref)) <= (np.log2(d) + 2) * 2.0 ** -24 * math.sqrt(d) * np.abs(X).max()
+    assert np.array_equal(fp8.transform_f32(X, None), X)
+
+
 def test_transform_spreads_a_single_outlier():
     d = 128
     x = np.zeros((1, d))
