@@ -108,54 +108,96 @@ struct Args {
   float inv_sqrt_d;
 };
 
-// Pass 1: one warp per (tensor, b, n, h) row.
+// Work split of passes 1 and 2a: CTA = (tensor, b, h, slice of kRowsPerCta tokens); its 8
+// warps take kUnroll rows at a time so that several row loads are in flight per warp.
+constexpr int kRowsPerCta = 512;
+constexpr int kUnroll = 4;
+
+struct Slice {
+  int t, b, h, n0, n1;
+};
+__device__ __forceinline__ Slice slice_of(const Args& a, int block) {
+  const int per_head = (a.N + kRowsPerCta - 1) / kRowsPerCta;
+  Slice s;
+  const int hs = block / per_head;  // (t, b, h) flattened
+  s.n0 = (block % per_head) * kRowsPerCta;
+  s.n1 = min(a.N, s.n0 + kRowsPerCta);
+  s.t = hs / (a.B * a.H);
+  s.b = (hs / a.H) % a.B;
+  s.h = hs % a.H;
+  return s;
+}
+__device__ __forceinline__ const __nv_bfloat16* src_of(const Args& a, int t) {
+  return t == 0 ? a.src_q : t == 1 ? a.src_k : a.src_v;
+}
+
+// Pass 1: per-head max |x| of the transformed Q, K and of V.
 template <int D>
 __global__ void __launch_bounds__(kThreads) amax_kernel(Args a) {
   constexpr int E = D / 32;
-  const int lane = threadIdx.x & 31;
-  const long long rows = static_cast<long long>(a.B) * a.N * a.H;
-  const long long warps = static_cast<long long>(gridDim.x) * (kThreads / 32);
-  for (long long w = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); w < 3 * rows; w += warps) {
-    const int t = static_cast<int>(w / rows);
-    const long long r = w % rows;  // (b, n, h) row-major
-    const int h = static_cast<int>(r % a.H);
-    const int b = static_cast<int>(r / (static_cast<long long>(a.N) * a.H));
-    float x[E];
-    load_row<E>((t == 0 ? a.src_q : t == 1 ? a.src_k : a.src_v) + r * D, lane, x);
-    if (t < 2 && a.signs) hadamard_row<E>(x, a.signs, lane, a.inv_sqrt_d);
-    float m = 0.f;
+  __shared__ float red[kThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const Slice s = slice_of(a, blockIdx.x);
+  const __nv_bfloat16* base = src_of(a, s.t) + (static_cast<size_t>(s.b) * a.N * a.H + s.h) * D;
+  const size_t row_stride = static_cast<size_t>(a.H) * D;
+  const bool xf = s.t < 2 && a.signs;
+  float m = 0.f;
+  for (int n = s.n0 + warp * kUnroll; n < s.n1; n += (kThreads / 32) * kUnroll) {
+    float x[kUnroll][E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(x[e]));
+    for (int u = 0; u < kUnroll; ++u)
+      if (n + u < s.n1) load_row<E>(base + (n + u) * row_stride, lane, x[u]);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (n + u >= s.n1) break;
+      if (xf) hadamard_row<E>(x[u], a.signs, lane, a.inv_sqrt_d);
+#pragma unroll
+      for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(x[u][e]));
+    }
+  }
+  m = warp_max(m);
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  if (warp == 0) {
+    m = lane < kThreads / 32 ? red[lane] : 0.f;
     m = warp_max(m);
-    if (lane == 0) atomicMax(a.amax + t * a.B * a.H + b * a.H + h, __float_as_uint(m));
+    if (lane == 0)
+      atomicMax(a.amax + s.t * a.B * a.H + s.b * a.H + s.h, __float_as_uint(m));
   }
 }
 
-// Pass 2a: Q and K codes, one warp per row; the first 3*B*H threads also publish the scales.
+// Pass 2a: Q and K codes (CTAs as in pass 1, tensors 0 and 1); CTA 0 also publishes the
+// scales of all three tensors.
 template <int D>
 __global__ void __launch_bounds__(kThreads) quant_qk_kernel(Args a) {
   constexpr int E = D / 32;
-  const int lane = threadIdx.x & 31;
-  const long long gtid = static_cast<long long>(blockIdx.x) * kThreads + threadIdx.x;
-  if (gtid < 3LL * a.B * a.H)
-    a.scales[gtid] = exp2i(scale_exp(__uint_as_float(a.amax[gtid])));
-  const long long rows = static_cast<long long>(a.B) * a.N * a.H;
-  const long long warps = static_cast<long long>(gridDim.x) * (kThreads / 32);
-  for (long long w = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); w < 2 * rows; w += warps) {
-    const int t = static_cast<int>(w / rows);
-    const long long r = w % rows;
-    const int h = static_cast<int>(r % a.H);
-    const int b = static_cast<int>(r / (static_cast<long long>(a.N) * a.H));
-    float x[E];
-    load_row<E>((t == 0 ? a.src_q : a.src_k) + r * D, lane, x);
-    if (a.signs) hadamard_row<E>(x, a.signs, lane, a.inv_sqrt_d);
-    const float inv = exp2i(-scale_exp(__uint_as_float(a.amax[t * a.B * a.H + b * a.H + h])));
-    uint8_t* out = (t == 0 ? a.dst_q : a.dst_k) + r * D + lane * E;
-    if constexpr (E == 4) {
-      const uint32_t lo = pack_e4m3x2(x[0] * inv, x[1] * inv), hi = pack_e4m3x2(x[2] * inv, x[3] * inv);
-      *reinterpret_cast<uint32_t*>(out) = lo | (hi << 16);
-    } else {
-      *reinterpret_cast<uint16_t*>(out) = pack_e4m3x2(x[0] * inv, x[1] * inv);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < 3 * a.B * a.H; i += kThreads)
+      a.scales[i] = exp2i(scale_exp(__uint_as_float(a.amax[i])));
+  const Slice s = slice_of(a, blockIdx.x);
+  const size_t head_off = (static_cast<size_t>(s.b) * a.N * a.H + s.h) * D;
+  const __nv_bfloat16* base = src_of(a, s.t) + head_off;
+  uint8_t* obase = (s.t == 0 ? a.dst_q : a.dst_k) + head_off + lane * E;
+  const size_t row_stride = static_cast<size_t>(a.H) * D;
+  const float inv = exp2i(-scale_exp(__uint_as_float(a.amax[s.t * a.B * a.H + s.b * a.H + s.h])));
+  for (int n = s.n0 + warp * kUnroll; n < s.n1; n += (kThreads / 32) * kUnroll) {
+    float x[kUnroll][E];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+      if (n + u < s.n1) load_row<E>(base + (n + u) * row_stride, lane, x[u]);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (n + u >= s.n1) break;
+      if (a.signs) hadamard_row<E>(x[u], a.signs, lane, a.inv_sqrt_d);
+      uint8_t* out = obase + (n + u) * row_stride;
+      if constexpr (E == 4) {
+        const uint32_t lo = pack_e4m3x2(x[u][0] * inv, x[u][1] * inv);
+        const uint32_t hi = pack_e4m3x2(x[u][2] * inv, x[u][3] * inv);
+        *reinterpret_cast<uint32_t*>(out) = lo | (hi << 16);
+      } else {
+        *reinterpret_cast<uint16_t*>(out) = static_cast<uint16_t>(pack_e4m3x2(x[u][0] * inv, x[u][1] * inv));
+      }
     }
   }
 }
@@ -222,13 +264,11 @@ static cudaError_t launch_t(const Fp8QuantArgs& p, cudaStream_t st) {
   a.inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
   cudaError_t e = cudaMemsetAsync(p.amax, 0, 3 * sizeof(uint32_t) * p.B * p.H, st);
   if (e != cudaSuccess) return e;
-  const long long rows = static_cast<long long>(p.B) * p.N * p.H;
-  const int grid_rows = static_cast<int>(std::min<long long>((3 * rows + 7) / 8, 148LL * 16));
-  amax_kernel<D><<<grid_rows, kThreads, 0, st>>>(a);
-  const long long need_scale_blocks = (3LL * p.B * p.H + kThreads - 1) / kThreads;
-  const int grid_q = static_cast<int>(
-      std::max<long long>(need_scale_blocks, std::min<long long>((2 * rows + 7) / 8, 148LL * 16)));
-  quant_qk_kernel<D><<<grid_q, kThreads, 0, st>>>(a);
+  const long long per_head = (p.N + kRowsPerCta - 1) / kRowsPerCta;
+  const long long heads = static_cast<long long>(p.B) * p.H;
+  if (3 * heads * per_head > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  amax_kernel<D><<<static_cast<int>(3 * heads * per_head), kThreads, 0, st>>>(a);
+  quant_qk_kernel<D><<<static_cast<int>(2 * heads * per_head), kThreads, 0, st>>>(a);
   const long long grid_v = static_cast<long long>(p.B) * p.H * ((a.npad + 127) / 128);
   if (grid_v > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   quant_vt_kernel<D><<<static_cast<int>(grid_v), kThreads, 0, st>>>(a);
