@@ -397,8 +397,11 @@ def run_reference(args, rank, world):
 
 def run_sweep(path: str, reps: int = 20, warmup: int = 3):
     """Times every workload of the benchmark sweep (forward-only configs: fa_fwd; forward +
-    backward configs: fa_fwd and fa_bwd separately) and writes one JSON line per workload
-    to `path`.  Median of `reps` CUDA-event timed launches after `warmup`."""
+    backward configs: fa_fwd, fa_bwd and fa_bwd_deterministic; decoding: fa_fwd_splitkv;
+    block-sparse masks against the dense forward; the FP8 forward and its operand
+    preparation) and writes one JSON line per workload to `path`.  Median of `reps`
+    CUDA-event timed launches after `warmup`."""
+    import numpy as np
     import torch
     from exact_io_aware_88_b200 import fa
     dev = torch.device("cuda", 0)
@@ -492,6 +495,44 @@ def run_sweep(path: str, reps: int = 20, warmup: int = 3):
             print(json.dumps(rec), file=sys.stderr)
             del q, k, v, o, lse, ws, t
             torch.cuda.empty_cache()
+        # Block-sparse forward: random block masks at several densities (diagonal blocks
+        # always kept), timed against the dense forward of the same problem.
+        B, N, H, d = 1, 16384, 16, 128
+        t = synthetic.draw(B, N, H, d, 1002, "bf16")
+        q, k, v = (t[n].to(dev) for n in ("q", "k", "v"))
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+        nt = N // 128
+        nb = fa.fa_fwd_block_sparse_workspace_bytes(B, H, N, d)
+        ws = torch.empty(nb, device=dev, dtype=torch.uint8)
+        rng = np.random.default_rng(7)
+        for causal in (False, True):
+            dense = lambda: fa.fa_fwd(q, k, v, o, lse, B, H, N, d, causal, 1.0 / math.sqrt(d), stream)
+            assert dense() == 0
+            dmed, _ = timed(dense)
+            for dens in (1.0, 0.5, 0.25, 0.1):
+                m = (rng.random((nt, nt)) < dens).astype(np.uint8)
+                np.fill_diagonal(m, 1)
+                if causal:
+                    m = np.tril(m)
+                mask = torch.from_numpy(m).to(dev)
+                act = int(m.sum())
+                tot = nt * (nt + 1) // 2 if causal else nt * nt
+                bs = lambda: fa.fa_fwd_block_sparse(q, k, v, o, lse, B, H, N, d, causal,
+                                                    1.0 / math.sqrt(d), mask, ws, nb, stream)
+                assert bs() == 0
+                med, best = timed(bs)
+                flops = 4.0 * B * H * 128 * 128 * d * act  # active blocks, counted whole
+                rec = {"workload": f"block_sparse:B{B}xN{N}xH{H}xd{d}" + ("-causal" if causal else "")
+                       + f"-density{act / tot:.2f}-bf16", "pass": "fwd_block_sparse",
+                       "ms": round(med, 4), "ms_best": round(best, 4),
+                       "tflops_active_blocks": round(flops / (med * 1e-3) / 1e12, 1),
+                       "dense_fa_fwd_ms": round(dmed, 4), "speedup_vs_dense": round(dmed / med, 3),
+                       "peak_source": peak_src}
+                out.write(json.dumps(rec) + "\n")
+                print(json.dumps(rec), file=sys.stderr)
+        del q, k, v, o, lse, ws, t
+        torch.cuda.empty_cache()
         # FP8 forward (E4M3 products, Hadamard-transformed Q and K): tensor-bound against the
         # bf16 measured peak x 2 (the nominal fp8 / bf16 ratio); the operand preparation
         # (fa_fp8_quantize) is timed separately and is HBM-bound.
