@@ -17,7 +17,8 @@
  *    カスタムモデルへの組み込み).  lse is a contiguous [B][H][N] fp32 array.
  *  - lse[b][h][i] = ln sum_j exp(scale * q_i . k_j) over the keys visible to query i
  *    (natural log, scale included).
- *  - Causal mask: key j is visible to query i iff j <= i.  Q and K have the same length N.
+ *  - Causal mask: key j is visible to query i iff j <= i.  Q and K have the same length N
+ *    (except fa_fwd_splitkv, whose causal rule aligns the last query with the last key).
  *  - scale is passed explicitly (1/sqrt(d) gives the textbook softmax); it must be a
  *    positive finite number (the kernels take each row maximum before scaling).
  *  - All tensor pointers are DEVICE pointers owned by the caller.  No entry point
