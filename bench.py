@@ -545,9 +545,18 @@ def run_sweep(path: str, reps: int = 20, warmup: int = 3):
             dense = lambda: fa.fa_fwd(q, k, v, o, lse, B, H, N, d, causal, 1.0 / math.sqrt(d), stream)
             assert dense() == 0
             dmed, _ = timed(dense)
-            for dens in (1.0, 0.5, 0.25, 0.1):
-                m = (rng.random((nt, nt)) < dens).astype(np.uint8)
-                np.fill_diagonal(m, 1)
+            # Random masks at four densities, then a structured one: a band of 8 key tiles
+            # ending at the diagonal plus the first key tile (local + global attention).
+            band = np.zeros((nt, nt), np.uint8)
+            for i in range(nt):
+                band[i, max(0, i - 7):i + 1] = 1
+                band[i, 0] = 1
+            for dens in (1.0, 0.5, 0.25, 0.1, "band8+global"):
+                if isinstance(dens, str):
+                    m = band.copy()
+                else:
+                    m = (rng.random((nt, nt)) < dens).astype(np.uint8)
+                    np.fill_diagonal(m, 1)
                 if causal:
                     m = np.tril(m)
                 mask = torch.from_numpy(m).to(dev)
@@ -558,8 +567,9 @@ def run_sweep(path: str, reps: int = 20, warmup: int = 3):
                 assert bs() == 0
                 med, best = timed(bs)
                 flops = 4.0 * B * H * 128 * 128 * d * act  # active blocks, counted whole
+                kind = dens if isinstance(dens, str) else "random"
                 rec = {"workload": f"block_sparse:B{B}xN{N}xH{H}xd{d}" + ("-causal" if causal else "")
-                       + f"-density{act / tot:.2f}-bf16", "pass": "fwd_block_sparse",
+                       + f"-{kind}-density{act / tot:.2f}-bf16", "pass": "fwd_block_sparse",
                        "ms": round(med, 4), "ms_best": round(best, 4),
                        "tflops_active_blocks": round(flops / (med * 1e-3) / 1e12, 1),
                        "dense_fa_fwd_ms": round(dmed, 4), "speedup_vs_dense": round(dmed / med, 3),

@@ -485,50 +485,49 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
   a.f16 = dtype == FA_DTYPE_FP16 ? 1 : 0;
   a.scale = scale;
   a.status = di.status;
-  a.block_mask = nullptr;
   return from_cuda(fa::launch_fwd_splitkv(a, static_cast<cudaStream_t>(stream)));
 }
 
 size_t fa_fwd_block_sparse_workspace_bytes(int B, int H, int N, int d) {
-  return fa_fwd_splitkv_workspace_bytes(B, H, N, N, d);
+  (void)B;
+  (void)H;
+  (void)d;
+  if (N < 1) return 0;
+  return round_up(static_cast<size_t>((N + 127) / 128) * 32 * sizeof(uint32_t), 256);
 }
 
 int fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                         int H, int N, int d, int causal, float scale, const uint8_t* block_mask,
                         void* workspace, size_t workspace_bytes, void* stream) {
   if (!q || !k || !v || !o || !lse || !block_mask) return FA_ERR_INVALID_ARG;
-  int rc = check_splitkv(B, H, N, N, d, causal, scale);
+  int rc = check_shape(B, H, N, d, scale);
   if (rc) return rc;
-  if ((N + 127) / 128 > 1024) return FA_ERR_UNSUPPORTED;  // per-row tile list limit
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if ((N + 127) / 128 > 1024) return FA_ERR_UNSUPPORTED;  // the kernel's per-tile bitmask limit
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return FA_ERR_MISALIGNED;
-  const size_t need = fa_fwd_block_sparse_workspace_bytes(B, H, N, d);
-  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
-  if (!aligned(workspace, 256)) return FA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < fa_fwd_block_sparse_workspace_bytes(B, H, N, d))
+    return FA_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return FA_ERR_MISALIGNED;
   DeviceInfo di;
   if ((rc = device_info(&di))) return rc;
-  fa::SplitKvArgs a;
+  fa::FwdArgs a;
   if ((rc = encode_bnhd(&a.tm_q, q, B, N, H, d)) || (rc = encode_bnhd(&a.tm_k, k, B, N, H, d)) ||
       (rc = encode_bnhd(&a.tm_v, v, B, N, H, d)))
     return rc;
-  splitkv_plan(B, H, N, N, &a.n_split, &a.tiles_per_split);
-  const size_t rows = static_cast<size_t>(a.n_split) * B * H * N;
-  char* ws = static_cast<char*>(workspace);
-  a.part_o = reinterpret_cast<float*>(ws);
-  a.part_lse = reinterpret_cast<float*>(ws + round_up(rows * d * sizeof(float), 256));
   a.o = o;
   a.lse = lse;
+  a.block_mask = block_mask;
+  a.mask_words = static_cast<uint32_t*>(workspace);
   a.B = B;
   a.H = H;
-  a.Nq = N;
-  a.Nk = N;
+  a.N = N;
   a.d = d;
   a.causal = causal ? 1 : 0;
-  a.f16 = 0;
   a.scale = scale;
   a.status = di.status;
-  a.block_mask = block_mask;
-  return from_cuda(fa::launch_fwd_splitkv(a, static_cast<cudaStream_t>(stream)));
+  a.num_sms = di.num_sms;
+  return from_cuda(fa::launch_fwd_block_sparse(a, static_cast<cudaStream_t>(stream)));
 }
 
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H,

@@ -76,7 +76,10 @@ struct Cfg {
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
   static constexpr int kBarBytes = 512;              // Bars (size checked below)
-  static constexpr int kSmemBytes = kOffBar + kBarBytes;  // base is 1024-aligned (checked)
+  // Block-sparse bitmasks: loader (2 tiles), MMA issuer (2), softmax warpgroup 0 and 1.
+  static constexpr int kOffMask = kOffBar + kBarBytes;
+  static constexpr int kMaskBytes = (2 + 2 + 8) * 32 * 4;  // + one copy per softmax warp
+  static constexpr int kSmemBytes = kOffMask + kMaskBytes;  // base is 1024-aligned (checked)
   static constexpr uint32_t kColO = 256;  // O_t at kColO + 128 t
 };
 
@@ -121,6 +124,68 @@ __device__ __forceinline__ int kv_tiles(int pair, int t, int kv_total) {
   return CAUSAL ? min(kv_total, 2 * pair + t + 1) : kv_total;
 }
 
+// Block-sparse activity of the pair's two query tiles as bitmasks in shared memory: bit j of
+// tile t is set iff key tile j is visible to it (kv_tiles) and the byte mask marks block
+// (query tile, j) active.  A query tile past the last one (odd tile count) has no bits.
+// Each role keeps its own copy (the roles work on different units at a time): the producer
+// and the MMA issuer one per tile, every softmax warp one of its own tile.
+constexpr int kMaskWords = 32;  // up to 1024 key tiles (N <= 131072)
+// Next set bit of a kMaskWords-word bitmask after j (-1: none); j = -1 gives the first.
+__device__ __forceinline__ int next_bit(const uint32_t* w, int j) {
+  int i = j + 1;
+  if (i >= 32 * kMaskWords) return -1;
+  int wi = i >> 5;
+  uint32_t bits = w[wi] & (0xffffffffu << (i & 31));
+  while (bits == 0u) {
+    if (++wi >= kMaskWords) return -1;
+    bits = w[wi];
+  }
+  return 32 * wi + __ffs(bits) - 1;
+}
+struct PairMask {
+  const uint32_t* w0;  // kMaskWords words per tile
+  const uint32_t* w1;
+  __device__ __forceinline__ int next(int t, int j) const { return next_bit(t ? w1 : w0, j); }
+  // Next key tile after j that either tile works on (-1: none).
+  __device__ __forceinline__ int next_any(int j) const {
+    const int a = next(0, j), b = next(1, j);
+    return a < 0 ? b : (b < 0 ? a : min(a, b));
+  }
+};
+// Packs the byte mask into kMaskWords bitmask words per query tile (run once per call, before
+// the attention kernel): bit j of tile qt is set iff key tile j is visible to qt and
+// mask[qt][j] != 0.  One thread per word.
+template <bool CAUSAL>
+__global__ void pack_mask_kernel(const uint8_t* __restrict__ mask, uint32_t* __restrict__ words,
+                                 int nq_tiles, int kv_total) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= nq_tiles * kMaskWords) return;
+  const int qt = i / kMaskWords, wi = i % kMaskWords;
+  const int nkv = CAUSAL ? min(kv_total, qt + 1) : kv_total;
+  const uint8_t* row = mask + static_cast<size_t>(qt) * kv_total;
+  uint32_t bits = 0u;
+#pragma unroll 4
+  for (int b = 0; b < 32; ++b) {
+    const int j = 32 * wi + b;
+    if (j < nkv && row[j] != 0) bits |= 1u << b;
+  }
+  words[i] = bits;
+}
+
+// Copies the pair's two tiles' words (tile 2*pair+t, zero for a tile past the last) into
+// this role's shared-memory copy: 2 x 128 bytes in 16-byte pieces.
+__device__ __forceinline__ void copy_pair_words(uint32_t* dst, const uint32_t* __restrict__ words,
+                                                int pair, int nq_tiles) {
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qt = 2 * pair + t;
+    const uint4* src = reinterpret_cast<const uint4*>(words + static_cast<size_t>(qt) * kMaskWords);
+    uint4* d4 = reinterpret_cast<uint4*>(dst + t * kMaskWords);
+#pragma unroll
+    for (int i = 0; i < kMaskWords / 4; ++i) d4[i] = qt < nq_tiles ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+  }
+}
+
 // Maximum of n values as a tree of 3-input max operations (depth log3 n).
 template <int n>
 __device__ __forceinline__ float tree_max(const float* v) {
@@ -141,12 +206,17 @@ __device__ __forceinline__ float tree_max(const float* v) {
 
 // F8: tm_q / tm_k map E4M3 [B][N][H][d], tm_v maps E4M3 V^T [B][H][d][Npad] (keys
 // contiguous), and scales[3][B*H] holds the per-head dequantisation scales of Q, K, V.
-template <int D, bool CAUSAL, bool F8>
+// SPARSE: mask_words (pack_mask_kernel's output, kMaskWords words per query tile) selects the
+// 128 x 128 blocks worked on (block-sparse attention); the loader streams the union of the
+// pair's active key tiles, each softmax warpgroup walks its own, and a query tile with none
+// gets O = 0, LSE = -inf.
+template <int D, bool CAUSAL, bool F8, bool SPARSE = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
-               float* __restrict__ lse, const float* __restrict__ scales, int B, int H, int N,
-               float scale_log2, int num_pairs, int* status, uint64_t timeout_ns) {
+               float* __restrict__ lse, const float* __restrict__ scales,
+               const uint32_t* __restrict__ mask_words, int B, int H, int N, float scale_log2,
+               int num_pairs, int* status, uint64_t timeout_ns) {
   using C = Cfg<D, F8>;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {  // 128-byte-swizzled tiles need a 1024-aligned base
@@ -223,7 +293,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float m = -INFINITY;  // running max of scale*log2(e)*s (possibly stale by < 2^8)
       float l = 0.f;
-      for (int j = 0; j < nkv; ++j) {
+      PairMask pm;
+      if constexpr (SPARSE) {
+        uint32_t* words = reinterpret_cast<uint32_t*>(smem + C::kOffMask) + (4 + warp) * kMaskWords;
+        const int qt = 2 * x.pair + t;
+        __syncwarp();  // every lane is done with the previous unit's words
+        words[lane] = qt < (N + BM - 1) / BM
+                          ? __ldg(mask_words + static_cast<size_t>(qt) * kMaskWords + lane)
+                          : 0u;
+        __syncwarp();
+        pm.w0 = pm.w1 = words;  // only tile t is asked for
+      }
+      for (int j = SPARSE ? pm.next(t, -1) : 0; SPARSE ? j >= 0 : j < nkv;
+           j = SPARSE ? pm.next(t, j) : j + 1) {
         // Decisions guarding warp-collective tcgen05.ld/st are made warp-uniform.
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], ns & 1, ab, status, timeout_ns));
         if (!ok) break;
@@ -336,8 +418,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bars->o_free[t]);  // the next unit's first PV may overwrite O_t now
       ++units;
+      // A query tile with no active block (block-sparse) has l = 0 and O_t holds nothing of
+      // this unit: O = 0, LSE = -inf.
+      const bool empty = SPARSE && l == 0.f;
+      if (empty) {
+#pragma unroll
+        for (int i = 0; i < D; ++i) o[i] = 0u;
+      }
       if (row < N) {
-        const float inv_l = out_mul / l;
+        const float inv_l = empty ? 0.f : out_mul / l;
         __nv_bfloat16* orow = out + ((static_cast<size_t>(b) * N + row) * H + h) * D;
 #pragma unroll
         for (int c8 = 0; c8 < D / 8; ++c8)
@@ -346,7 +435,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               pack_bf16x2(__uint_as_float(o[8 * c8 + 2]) * inv_l, __uint_as_float(o[8 * c8 + 3]) * inv_l),
               pack_bf16x2(__uint_as_float(o[8 * c8 + 4]) * inv_l, __uint_as_float(o[8 * c8 + 5]) * inv_l),
               pack_bf16x2(__uint_as_float(o[8 * c8 + 6]) * inv_l, __uint_as_float(o[8 * c8 + 7]) * inv_l));
-        lse[static_cast<size_t>(x.bh) * N + row] = (m + __log2f(l)) * 0.69314718055994531f;
+        lse[static_cast<size_t>(x.bh) * N + row] =
+            empty ? -INFINITY : (m + __log2f(l)) * 0.69314718055994531f;
       }
     }
   } else {
@@ -377,7 +467,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                           c * C::kChunkElems, h, (2 * x.pair + t) * BM, b, pol_q);
           ++units;
           const int nkv = kv_tiles<CAUSAL>(x.pair, 1, kv_total);
-          for (int j = 0; j < nkv; ++j, ++g) {
+          PairMask pm;
+          if constexpr (SPARSE) {
+            uint32_t* words = reinterpret_cast<uint32_t*>(smem + C::kOffMask);
+            copy_pair_words(words, mask_words, x.pair, (N + BM - 1) / BM);
+            pm.w0 = words;
+            pm.w1 = words + kMaskWords;
+          }
+          for (int j = SPARSE ? pm.next_any(-1) : 0; SPARSE ? j >= 0 : j < nkv;
+               j = SPARSE ? pm.next_any(j) : j + 1, ++g) {
             const int s = g % C::kStages;
             const uint32_t ph = ((g / C::kStages) - 1) & 1;
             if (g >= C::kStages &&
@@ -458,66 +556,195 @@ __global__ void __launch_bounds__(kThreads, 1)
                       (!first || kk > 0) ? 1u : 0u);
           }
         };
-        for (int r = 0; ok; ++r) {
-          const int u = unit_of_round(r, G);
-          if (u >= num_units) break;
-          const Unit x = decode_unit<CAUSAL>(u, BH, num_pairs);
-          const int nkv0 = kv_tiles<CAUSAL>(x.pair, 0, kv_total);
-          const int nkv1 = kv_tiles<CAUSAL>(x.pair, 1, kv_total);
-          if (!(ok = mbar_wait(&bars->q_full, units & 1, ab, status, timeout_ns))) break;
-          {  // prologue: S0(0), S1(0)
-            const int s = g % C::kStages;
-            if (!(ok = mbar_wait(&bars->k_full[s], (g / C::kStages) & 1, ab, status, timeout_ns)))
-              break;
-            tc_fence_after();
-            issue_s(0, s);
-            issue_s(1, s);
-            umma_commit(&bars->k_empty[s]);
-            if (nkv1 == 1) umma_commit(&bars->q_empty);  // last S products of this unit
-          }
-          for (int j = 0; ok && j < nkv1; ++j) {
-            const int s = (g + j) % C::kStages;
-            const int s1 = (g + j + 1) % C::kStages;
-            const bool more = j + 1 < nkv1;
-            if (!(ok = mbar_wait(&bars->v_full[s], ((g + j) / C::kStages) & 1, ab, status,
-                                 timeout_ns)))
-              break;
-            if (more && !(ok = mbar_wait(&bars->k_full[s1], ((g + j + 1) / C::kStages) & 1, ab,
-                                         status, timeout_ns)))
-              break;
-            if (j < nkv0) {  // tile 0: PV0(j), S0(j+1)
-              if (j == 0 && units > 0 &&
-                  !(ok = mbar_wait(&bars->o_free[0], (units - 1) & 1, ab, status, timeout_ns)))
+        if constexpr (SPARSE) {
+          // Block-sparse issue order.  Key tiles come in the union order of the two query
+          // tiles' active lists (the loader's ring order).  At each such key tile j: first
+          // any S_t(j) still owed (deferred because j was not the next ring tile when
+          // PV_t(previous) was issued), then for every tile active at j: PV_t(j) followed,
+          // when t's next active tile is also the next ring tile, by S_t(next) at once (the
+          // dense order).  A K stage is released once every S on it has been issued.
+          const int nq_tiles = (N + BM - 1) / BM;
+          for (int r = 0; ok; ++r) {
+            const int u = unit_of_round(r, G);
+            if (u >= num_units) break;
+            const Unit x = decode_unit<CAUSAL>(u, BH, num_pairs);
+            PairMask pm;
+            {
+              uint32_t* words = reinterpret_cast<uint32_t*>(smem + C::kOffMask) + 2 * kMaskWords;
+              copy_pair_words(words, mask_words, x.pair, nq_tiles);
+              pm.w0 = words;
+              pm.w1 = words + kMaskWords;
+            }
+            if (!(ok = mbar_wait(&bars->q_full, units & 1, ab, status, timeout_ns))) break;
+            // Per-tile state, kept in scalars (t is a compile-time constant below).
+            int cur0 = pm.next(0, -1), cur1 = pm.next(1, -1);  // each tile's next key tile
+            bool sd0 = false, sd1 = false;                      // S_t(cur_t) issued
+            bool fp0 = true, fp1 = true;                        // first PV of the unit
+            bool ls0 = cur0 < 0, ls1 = cur1 < 0;                // no S left to issue for t
+            bool q_released = false;
+            auto release_q = [&]() {
+              if (!q_released && ls0 && ls1) {
+                umma_commit(&bars->q_empty);
+                q_released = true;
+              }
+            };
+            if (cur0 < 0) umma_commit(&bars->o_done[0]);  // nothing accumulated: done
+            if (cur1 < 0) umma_commit(&bars->o_done[1]);
+            int j = pm.next_any(-1);
+            int gu = g;  // ring position of key tile j
+            if (j >= 0) {
+              const int s = gu % C::kStages;
+              if (!(ok = mbar_wait(&bars->k_full[s], (gu / C::kStages) & 1, ab, status,
+                                   timeout_ns)))
                 break;
-              if (!(ok = mbar_wait(&bars->p_full[0], np[0] & 1, ab, status, timeout_ns))) break;
-              ++np[0];
               tc_fence_after();
-              issue_pv(0, s, j == 0);
-              if (j + 1 < nkv0) {
-                issue_s(0, s1);
+              if (cur0 == j) {
+                issue_s(0, s);
+                sd0 = true;
+                ls0 = pm.next(0, j) < 0;
+              }
+              if (cur1 == j) {
+                issue_s(1, s);
+                sd1 = true;
+                ls1 = pm.next(1, j) < 0;
+              }
+              umma_commit(&bars->k_empty[s]);  // every tile active at j is served
+            }
+            release_q();
+            while (ok && j >= 0) {
+              const int s = gu % C::kStages;
+              const int sn = (gu + 1) % C::kStages;
+              // Everything this step needs from the masks, before any wait.
+              const bool on0 = cur0 == j, on1 = cur1 == j;
+              const int nt0 = on0 ? pm.next(0, j) : cur0;
+              const int nt1 = on1 ? pm.next(1, j) : cur1;
+              const int jn = (nt0 < 0) ? nt1 : ((nt1 < 0) ? nt0 : min(nt0, nt1));
+              const bool last0 = nt0 < 0 || pm.next(0, nt0) < 0;
+              const bool last1 = nt1 < 0 || pm.next(1, nt1) < 0;
+              // S owed on j (its K stage is still held for it).
+              const bool owe0 = on0 && !sd0, owe1 = on1 && !sd1;
+              if (owe0 || owe1) {
+                tc_fence_after();
+                if (owe0) {
+                  issue_s(0, s);
+                  ls0 = !(nt0 >= 0);
+                }
+                if (owe1) {
+                  issue_s(1, s);
+                  ls1 = !(nt1 >= 0);
+                }
+                umma_commit(&bars->k_empty[s]);
+                release_q();
+              }
+              if (!(ok = mbar_wait(&bars->v_full[s], (gu / C::kStages) & 1, ab, status,
+                                   timeout_ns)))
+                break;
+              if (jn >= 0 && !(ok = mbar_wait(&bars->k_full[sn], ((gu + 1) / C::kStages) & 1, ab,
+                                               status, timeout_ns)))
+                break;
+              // The V stage is released right after the last PV that reads it, before that
+              // tile's next S, so that its reload is not held up by the S product.
+              auto pv_then_next_s = [&](auto tc, bool on, bool& fp, int& cur, bool& sd, bool& ls,
+                                        int nt, bool last, bool last_pv) -> bool {
+                constexpr int t = decltype(tc)::value;
+                if (!on) return true;
+                if (fp && units > 0 &&
+                    !mbar_wait(&bars->o_free[t], (units - 1) & 1, ab, status, timeout_ns))
+                  return false;
+                if (!mbar_wait(&bars->p_full[t], np[t] & 1, ab, status, timeout_ns)) return false;
+                ++np[t];
+                tc_fence_after();
+                issue_pv(t, s, fp);
+                if (last_pv) umma_commit(&bars->v_empty[s]);
+                fp = false;
+                cur = nt;
+                sd = false;
+                if (nt < 0) {
+                  umma_commit(&bars->o_done[t]);
+                } else if (nt == jn) {
+                  issue_s(t, sn);
+                  sd = true;
+                  ls = last;
+                }
+                return true;
+              };
+              if (!(ok = pv_then_next_s(std::integral_constant<int, 0>{}, on0, fp0, cur0, sd0, ls0,
+                                        nt0, last0, !on1)))
+                break;
+              if (!(ok = pv_then_next_s(std::integral_constant<int, 1>{}, on1, fp1, cur1, sd1, ls1,
+                                        nt1, last1, true)))
+                break;
+              if (jn >= 0 && !((cur0 == jn && !sd0) || (cur1 == jn && !sd1)))
+                umma_commit(&bars->k_empty[sn]);  // no S owed on jn: its K stage is free
+              release_q();
+              j = jn;
+              ++gu;
+            }
+            g = gu;
+            ++units;
+          }
+        } else {
+          for (int r = 0; ok; ++r) {
+            const int u = unit_of_round(r, G);
+            if (u >= num_units) break;
+            const Unit x = decode_unit<CAUSAL>(u, BH, num_pairs);
+            const int nkv0 = kv_tiles<CAUSAL>(x.pair, 0, kv_total);
+            const int nkv1 = kv_tiles<CAUSAL>(x.pair, 1, kv_total);
+            if (!(ok = mbar_wait(&bars->q_full, units & 1, ab, status, timeout_ns))) break;
+            {  // prologue: S0(0), S1(0)
+              const int s = g % C::kStages;
+              if (!(ok = mbar_wait(&bars->k_full[s], (g / C::kStages) & 1, ab, status, timeout_ns)))
+                break;
+              tc_fence_after();
+              issue_s(0, s);
+              issue_s(1, s);
+              umma_commit(&bars->k_empty[s]);
+              if (nkv1 == 1) umma_commit(&bars->q_empty);  // last S products of this unit
+            }
+            for (int j = 0; ok && j < nkv1; ++j) {
+              const int s = (g + j) % C::kStages;
+              const int s1 = (g + j + 1) % C::kStages;
+              const bool more = j + 1 < nkv1;
+              if (!(ok = mbar_wait(&bars->v_full[s], ((g + j) / C::kStages) & 1, ab, status,
+                                   timeout_ns)))
+                break;
+              if (more && !(ok = mbar_wait(&bars->k_full[s1], ((g + j + 1) / C::kStages) & 1, ab,
+                                           status, timeout_ns)))
+                break;
+              if (j < nkv0) {  // tile 0: PV0(j), S0(j+1)
+                if (j == 0 && units > 0 &&
+                    !(ok = mbar_wait(&bars->o_free[0], (units - 1) & 1, ab, status, timeout_ns)))
+                  break;
+                if (!(ok = mbar_wait(&bars->p_full[0], np[0] & 1, ab, status, timeout_ns))) break;
+                ++np[0];
+                tc_fence_after();
+                issue_pv(0, s, j == 0);
+                if (j + 1 < nkv0) {
+                  issue_s(0, s1);
+                } else {
+                  umma_commit(&bars->o_done[0]);
+                }
+              }
+              // tile 1: PV1(j), S1(j+1)
+              if (j == 0 && units > 0 &&
+                  !(ok = mbar_wait(&bars->o_free[1], (units - 1) & 1, ab, status, timeout_ns)))
+                break;
+              if (!(ok = mbar_wait(&bars->p_full[1], np[1] & 1, ab, status, timeout_ns))) break;
+              ++np[1];
+              tc_fence_after();
+              issue_pv(1, s, j == 0);
+              umma_commit(&bars->v_empty[s]);
+              if (more) {
+                issue_s(1, s1);
+                umma_commit(&bars->k_empty[s1]);
+                if (j + 2 == nkv1) umma_commit(&bars->q_empty);  // last S products of this unit
               } else {
-                umma_commit(&bars->o_done[0]);
+                umma_commit(&bars->o_done[1]);
               }
             }
-            // tile 1: PV1(j), S1(j+1)
-            if (j == 0 && units > 0 &&
-                !(ok = mbar_wait(&bars->o_free[1], (units - 1) & 1, ab, status, timeout_ns)))
-              break;
-            if (!(ok = mbar_wait(&bars->p_full[1], np[1] & 1, ab, status, timeout_ns))) break;
-            ++np[1];
-            tc_fence_after();
-            issue_pv(1, s, j == 0);
-            umma_commit(&bars->v_empty[s]);
-            if (more) {
-              issue_s(1, s1);
-              umma_commit(&bars->k_empty[s1]);
-              if (j + 2 == nkv1) umma_commit(&bars->q_empty);  // last S products of this unit
-            } else {
-              umma_commit(&bars->o_done[1]);
-            }
+            g += nkv1;
+            ++units;
           }
-          g += nkv1;
-          ++units;
         }
         // Drain every MMA this thread issued before TMEM is released.
         umma_commit(&bars->drain);
@@ -536,10 +763,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool CAUSAL, bool F8 = false>
+template <int D, bool CAUSAL, bool F8 = false, bool SPARSE = false>
 static cudaError_t launch_t(const FwdArgs& a, cudaStream_t st) {
   using C = Cfg<D, F8>;
-  auto kern = fwd_kernel<D, CAUSAL, F8>;
+  auto kern = fwd_kernel<D, CAUSAL, F8, SPARSE>;
   // The setmaxnreg split assumes the kernel launches with exactly kRegsLaunch registers per
   // thread; with fewer, the softmax warpgroups' increase could never be satisfied.
   cudaFuncAttributes fa_attr;
@@ -555,8 +782,8 @@ static cudaError_t launch_t(const FwdArgs& a, cudaStream_t st) {
   const float scale_log2 = a.scale * 1.4426950408889634f;
   kern<<<grid, kThreads, C::kSmemBytes, st>>>(a.tm_q, a.tm_k, a.tm_v,
                                               static_cast<__nv_bfloat16*>(a.o), a.lse, a.scales,
-                                              a.B, a.H, a.N, scale_log2, num_pairs, a.status,
-                                              kDefaultWaitTimeoutNs);
+                                              a.mask_words, a.B, a.H, a.N, scale_log2, num_pairs,
+                                              a.status, kDefaultWaitTimeoutNs);
   return cudaGetLastError();
 }
 
@@ -565,6 +792,22 @@ static cudaError_t launch_t(const FwdArgs& a, cudaStream_t st) {
 cudaError_t launch_fwd_sm100(const FwdArgs& a, cudaStream_t s) {
   if (a.d == 64) return a.causal ? fwd::launch_t<64, true>(a, s) : fwd::launch_t<64, false>(a, s);
   return a.causal ? fwd::launch_t<128, true>(a, s) : fwd::launch_t<128, false>(a, s);
+}
+
+cudaError_t launch_fwd_block_sparse(const FwdArgs& a, cudaStream_t s) {
+  const int nq = (a.N + fwd::BM - 1) / fwd::BM, nk = (a.N + fwd::BN - 1) / fwd::BN;
+  const int n = nq * fwd::kMaskWords;
+  if (a.causal)
+    fwd::pack_mask_kernel<true><<<(n + 255) / 256, 256, 0, s>>>(a.block_mask, a.mask_words, nq, nk);
+  else
+    fwd::pack_mask_kernel<false><<<(n + 255) / 256, 256, 0, s>>>(a.block_mask, a.mask_words, nq, nk);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (a.d == 64)
+    return a.causal ? fwd::launch_t<64, true, false, true>(a, s)
+                    : fwd::launch_t<64, false, false, true>(a, s);
+  return a.causal ? fwd::launch_t<128, true, false, true>(a, s)
+                  : fwd::launch_t<128, false, false, true>(a, s);
 }
 
 cudaError_t launch_fwd_fp8(const FwdArgs& a, cudaStream_t s) {

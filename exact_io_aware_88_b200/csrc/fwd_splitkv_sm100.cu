@@ -39,7 +39,6 @@ constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kMaxListTiles = 1024;        // block-sparse: key tiles per row of the mask
 
 template <int D>
 struct Cfg {
@@ -51,8 +50,7 @@ struct Cfg {
   static constexpr int kOffK = kOffQ + kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kOffList = kOffBar + 256;    // active key tiles (block-sparse)
-  static constexpr int kSmemBytes = kOffList + 2 * kMaxListTiles;  // base 1024-aligned (checked)
+  static constexpr int kSmemBytes = kOffBar + 256;  // base is 1024-aligned (checked)
 };
 
 struct Bars {
@@ -62,8 +60,7 @@ struct Bars {
   uint32_t tmem_base;
   Abort abort;
 };
-// The block-sparse tile count sits at byte 248 of the 256-byte barrier region.
-static_assert(sizeof(Bars) <= 248, "barrier block larger than its shared-memory region");
+static_assert(sizeof(Bars) <= 256, "barrier block larger than its shared-memory region");
 
 template <bool F16>
 __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
@@ -81,17 +78,13 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_m
              : idesc_bf16_f32(M, N, a_mn, b_mn);
 }
 
-// SPARSE: block-sparse attention ("FlashAttention――GPUメモリの読み書きを減らし、注意機構を
-// 正確なまま高速・省メモリに", section 手法): only the key tiles whose entry in the 128x128
-// block mask (row = query tile) is set are loaded and computed; the slices of the split then
-// index that list of active tiles.
-template <int D, bool CAUSAL, bool F16, bool SPARSE>
+template <int D, bool CAUSAL, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     splitkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, float* __restrict__ part_o,
                    float* __restrict__ part_lse, int H, int Nq, int Nk, int n_split,
-                   int tiles_per_split, int num_qtiles, int BH, float scale_log2,
-                   const uint8_t* __restrict__ block_mask, int* status, uint64_t timeout_ns) {
+                   int tiles_per_split, int num_qtiles, int BH, float scale_log2, int* status,
+                   uint64_t timeout_ns) {
   using C = Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
@@ -111,18 +104,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int off = Nk - Nq;  // causal alignment of the last query with the last key
   const int last_key = CAUSAL ? min(Nk - 1, q0 + BM - 1 + off) : Nk - 1;
   const int nvis = last_key / BN + 1;  // key tiles any row of this query tile can see
-  int16_t* list = reinterpret_cast<int16_t*>(smem + C::kOffList);
-  int* list_len = reinterpret_cast<int*>(smem + C::kOffBar + 248);
+  const int j_begin = split * tiles_per_split;
+  const int j_end = min(nvis, j_begin + tiles_per_split);
+  const int nkv = max(0, j_end - j_begin);
 
   if (threadIdx.x == 0) {
-    if constexpr (SPARSE) {
-      const int nk_tiles = (Nk + BN - 1) / BN;
-      const uint8_t* mrow = block_mask + static_cast<size_t>(qt) * nk_tiles;
-      int cnt = 0;
-      for (int j = 0; j < nvis; ++j)
-        if (mrow[j]) list[cnt++] = static_cast<int16_t>(j);
-      *list_len = cnt;
-    }
     mbar_init(&bars->q_full, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
@@ -148,11 +134,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = bars->tmem_base;
   Abort* ab = &bars->abort;
-  const int nact = SPARSE ? *list_len : nvis;  // key tiles this query tile visits
-  const int j_begin = split * tiles_per_split;
-  const int j_end = min(nact, j_begin + tiles_per_split);
-  const int nkv = max(0, j_end - j_begin);
-  auto tile_of = [&](int n) -> int { return SPARSE ? list[j_begin + n] : j_begin + n; };
   uint8_t* sQ = smem + C::kOffQ;
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
@@ -170,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(sQ + c * C::kChunkBytes, &tm_q, &bars->q_full, c * 64, h, q0, b, pol_q);
       int issued = 0;
       for (int n = 0; n < nkv; ++n) {
-        const int j = tile_of(n);
+        const int j = j_begin + n;
         const int s = n % C::kStages;
         if (n >= C::kStages &&
             !mbar_wait(&bars->kv_empty[s], ((n / C::kStages) - 1) & 1, ab, status, timeout_ns))
@@ -259,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 64; ++i) sv[64 * c + i] = __uint_as_float(u[i]);
         }
-        const int k0 = tile_of(n) * BN;
+        const int k0 = (j_begin + n) * BN;
         const int lim = min(CAUSAL ? row + off : Nk - 1, Nk - 1) - k0;  // last visible column
         if (__any_sync(0xffffffffu, lim < BN - 1)) {
 #pragma unroll
@@ -398,10 +379,10 @@ __global__ void __launch_bounds__(256)
   if (part == 0) lse[rowid] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
 }
 
-template <int D, bool CAUSAL, bool F16, bool SPARSE>
+template <int D, bool CAUSAL, bool F16>
 static cudaError_t launch_t(const SplitKvArgs& a, cudaStream_t st) {
   using C = Cfg<D>;
-  auto kern = splitkv_kernel<D, CAUSAL, F16, SPARSE>;
+  auto kern = splitkv_kernel<D, CAUSAL, F16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -411,7 +392,7 @@ static cudaError_t launch_t(const SplitKvArgs& a, cudaStream_t st) {
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, st>>>(
       a.tm_q, a.tm_k, a.tm_v, a.part_o, a.part_lse, a.H, a.Nq, a.Nk, a.n_split,
-      a.tiles_per_split, num_qtiles, BH, a.scale * 1.4426950408889634f, a.block_mask, a.status,
+      a.tiles_per_split, num_qtiles, BH, a.scale * 1.4426950408889634f, a.status,
       kDefaultWaitTimeoutNs);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -426,22 +407,15 @@ static cudaError_t launch_t(const SplitKvArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <bool SPARSE>
-static cudaError_t dispatch(const SplitKvArgs& a, cudaStream_t s) {
-  if (a.d == 64) {
-    if (a.f16)
-      return a.causal ? launch_t<64, true, true, SPARSE>(a, s) : launch_t<64, false, true, SPARSE>(a, s);
-    return a.causal ? launch_t<64, true, false, SPARSE>(a, s) : launch_t<64, false, false, SPARSE>(a, s);
-  }
-  if (a.f16)
-    return a.causal ? launch_t<128, true, true, SPARSE>(a, s) : launch_t<128, false, true, SPARSE>(a, s);
-  return a.causal ? launch_t<128, true, false, SPARSE>(a, s) : launch_t<128, false, false, SPARSE>(a, s);
-}
-
 }  // namespace splitkv
 
 cudaError_t launch_fwd_splitkv(const SplitKvArgs& a, cudaStream_t s) {
-  return a.block_mask ? splitkv::dispatch<true>(a, s) : splitkv::dispatch<false>(a, s);
+  if (a.d == 64) {
+    if (a.f16) return a.causal ? splitkv::launch_t<64, true, true>(a, s) : splitkv::launch_t<64, false, true>(a, s);
+    return a.causal ? splitkv::launch_t<64, true, false>(a, s) : splitkv::launch_t<64, false, false>(a, s);
+  }
+  if (a.f16) return a.causal ? splitkv::launch_t<128, true, true>(a, s) : splitkv::launch_t<128, false, true>(a, s);
+  return a.causal ? splitkv::launch_t<128, true, false>(a, s) : splitkv::launch_t<128, false, false>(a, s);
 }
 
 }  // namespace fa

@@ -19,6 +19,8 @@ struct FwdArgs {
   void* o;
   float* lse;
   const float* scales = nullptr;  // 8-bit path: [3][B*H] dequantisation scales
+  const uint8_t* block_mask = nullptr;  // block-sparse: [ceil(N/128)][ceil(N/128)] bytes
+  uint32_t* mask_words = nullptr;       // block-sparse: packed bitmasks (workspace)
   int B, H, N, d, causal;
   float scale;
   int* status;
@@ -46,7 +48,6 @@ struct SplitKvArgs {
   float* lse;                    // [B][H][Nq]
   float* part_o;                 // [n_split][B*H][Nq][d] fp32 workspace
   float* part_lse;               // [n_split][B*H][Nq] fp32 workspace
-  const uint8_t* block_mask;     // block-sparse: [ceil(Nq/128)][ceil(Nk/128)] or null
   int B, H, Nq, Nk, d, causal, f16;
   int n_split, tiles_per_split;
   float scale;
@@ -55,6 +56,7 @@ struct SplitKvArgs {
 
 cudaError_t launch_fwd_sm100(const FwdArgs& a, cudaStream_t s);
 cudaError_t launch_fwd_fp8(const FwdArgs& a, cudaStream_t s);
+cudaError_t launch_fwd_block_sparse(const FwdArgs& a, cudaStream_t s);
 
 struct Fp8QuantArgs {
   const void *q, *k, *v;  // [B][N][H][d] bf16

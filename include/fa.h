@@ -156,11 +156,15 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
  * ("FlashAttention――GPUメモリの読み書きを減らし、注意機構を正確なまま高速・省メモリに",
  * section 手法): key j is visible to query i iff block_mask[i/128][j/128] != 0 (and, if
  * causal, j <= i); masked 128x128 blocks are neither loaded nor computed.
- *   q, k, v, o : [B][N][H][d] bf16; lse : [B][H][N] fp32; d in {64, 128}; N <= 131072.
+ *   q, k, v, o : [B][N][H][d] bf16; lse : [B][H][N] fp32; d in {64, 128}; N <= 131072
+ *   (larger: FA_ERR_UNSUPPORTED).
  *   block_mask : DEVICE pointer, [ceil(N/128)][ceil(N/128)] bytes, shared by all batches and
  *                heads.
  *   A query that sees no key at all gets O = 0 and lse = -inf.
- *   workspace : >= fa_fwd_block_sparse_workspace_bytes(B, H, N, d), 256-byte aligned. */
+ *   Runs on the forward kernel of fa_fwd, which streams, for each pair of query tiles, the
+ *   union of their active key tiles.
+ *   workspace : >= fa_fwd_block_sparse_workspace_bytes(B, H, N, d) bytes (the mask packed
+ *   into 128 bytes of bits per query tile), 16-byte aligned, caller-owned. */
 size_t fa_fwd_block_sparse_workspace_bytes(int B, int H, int N, int d);
 int fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
                         int B, int H, int N, int d, int causal, float scale,

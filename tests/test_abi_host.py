@@ -116,6 +116,20 @@ def test_fp8_entry_points_reject_bad_arguments_without_launching(fa):
     assert q(signs=A16 + 2) == fa.FA_ERR_MISALIGNED
 
 
+def test_block_sparse_workspace_is_the_packed_mask(fa):
+    # 128 bytes of bits per 128-row query tile, rounded up to 256 bytes.
+    assert fa.fa_fwd_block_sparse_workspace_bytes(2, 4, 4096, 128) == 32 * 128
+    assert fa.fa_fwd_block_sparse_workspace_bytes(1, 1, 1000, 64) == 8 * 128
+    assert fa.fa_fwd_block_sparse_workspace_bytes(1, 1, 100, 64) == 256
+    base = [A16] * 5
+    call = lambda ws, wsb, N=1000: fa.fa_fwd_block_sparse(*base, 1, 2, N, 128, 0, 0.1, A16, ws,
+                                                          wsb, stream=0)
+    assert call(None, 4096) == fa.FA_ERR_WORKSPACE
+    assert call(A16, 1023) == fa.FA_ERR_WORKSPACE
+    assert call(A16 + 8, 1024) == fa.FA_ERR_MISALIGNED
+    assert call(A16, 1 << 20, N=131073) == fa.FA_ERR_UNSUPPORTED
+
+
 def test_debug_entry_points_reject_bad_arguments(fa):
     assert fa.fa_debug_umma_tile(A16, A16, A16, 96, 64, 0, stream=0) == fa.FA_ERR_UNSUPPORTED
     assert fa.fa_debug_umma_tile(A16, A16, A16, 64, 64, 3, stream=0) == fa.FA_ERR_UNSUPPORTED

@@ -120,3 +120,21 @@ def test_block_sparse_all_ones_equals_dense_and_empty_rows(fa):
     m = np.eye(5, dtype=np.uint8)
     m[2, 2] = 0  # block row 2 sees nothing: O = 0, lse = -inf
     _bs_case(fa, 1, N, 2, d, False, m, 6101)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_sparse_interleaved_and_odd_tile_counts(fa, d, causal):
+    """Masks that make the two query tiles of a pair take turns (tile 2p on even key tiles,
+    tile 2p+1 on odd ones, so most of each tile's next products wait for a later key tile),
+    an odd number of query tiles (the last pair has one tile), and a pair with one tile
+    empty."""
+    N = 1100  # 9 query tiles
+    nt = (N + 127) // 128
+    m = np.zeros((nt, nt), np.uint8)
+    for i in range(nt):
+        m[i, (i % 2)::2] = 1
+        m[i, i] = 1
+    m[3, :] = 0  # tile 3 sees nothing: O = 0, lse = -inf (its pair partner is tile 2)
+    _bs_case(fa, 1, N, 3, d, causal, m, 6200 + d)
+
