@@ -130,27 +130,31 @@ __device__ __forceinline__ int kv_tiles(int pair, int t, int kv_total) {
 // Each role keeps its own copy (the roles work on different units at a time): the producer
 // and the MMA issuer one per tile, every softmax warp one of its own tile.
 constexpr int kMaskWords = 32;  // up to 1024 key tiles (N <= 131072)
-// Next set bit of a kMaskWords-word bitmask after j (-1: none); j = -1 gives the first.
-__device__ __forceinline__ int next_bit(const uint32_t* w, int j) {
-  int i = j + 1;
-  if (i >= 32 * kMaskWords) return -1;
-  int wi = i >> 5;
-  uint32_t bits = w[wi] & (0xffffffffu << (i & 31));
-  while (bits == 0u) {
-    if (++wi >= kMaskWords) return -1;
-    bits = w[wi];
+// Walks the set bits of one tile's bitmask in order, one word cached in a register.
+struct BitIter {
+  const uint32_t* w;
+  int wi;
+  uint32_t bits;
+  __device__ __forceinline__ void init(const uint32_t* words) {
+    w = words;
+    wi = 0;
+    bits = words[0];
   }
-  return 32 * wi + __ffs(bits) - 1;
-}
+  // Returns the next set bit (consuming it), or -1 when none is left.
+  __device__ __forceinline__ int pop() {
+    while (bits == 0u) {
+      if (++wi >= kMaskWords) return -1;
+      bits = w[wi];
+    }
+    const int b = __ffs(bits) - 1;
+    bits &= bits - 1u;
+    return 32 * wi + b;
+  }
+};
+
 struct PairMask {
   const uint32_t* w0;  // kMaskWords words per tile
   const uint32_t* w1;
-  __device__ __forceinline__ int next(int t, int j) const { return next_bit(t ? w1 : w0, j); }
-  // Next key tile after j that either tile works on (-1: none).
-  __device__ __forceinline__ int next_any(int j) const {
-    const int a = next(0, j), b = next(1, j);
-    return a < 0 ? b : (b < 0 ? a : min(a, b));
-  }
 };
 // Packs the byte mask into kMaskWords bitmask words per query tile (run once per call, before
 // the attention kernel): bit j of tile qt is set iff key tile j is visible to qt and
@@ -304,8 +308,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         pm.w0 = pm.w1 = words;  // only tile t is asked for
       }
-      for (int j = SPARSE ? pm.next(t, -1) : 0; SPARSE ? j >= 0 : j < nkv;
-           j = SPARSE ? pm.next(t, j) : j + 1) {
+      BitIter it;
+      if constexpr (SPARSE) it.init(pm.w0);
+      for (int j = SPARSE ? it.pop() : 0; SPARSE ? j >= 0 : j < nkv; j = SPARSE ? it.pop() : j + 1) {
         // Decisions guarding warp-collective tcgen05.ld/st are made warp-uniform.
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], ns & 1, ab, status, timeout_ns));
         if (!ok) break;
@@ -474,8 +479,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             pm.w0 = words;
             pm.w1 = words + kMaskWords;
           }
-          for (int j = SPARSE ? pm.next_any(-1) : 0; SPARSE ? j >= 0 : j < nkv;
-               j = SPARSE ? pm.next_any(j) : j + 1, ++g) {
+          BitIter it0, it1;
+          int h0 = -1, h1 = -1;  // next active key tile of each tile (sparse)
+          if constexpr (SPARSE) {
+            it0.init(pm.w0);
+            it1.init(pm.w1);
+            h0 = it0.pop();
+            h1 = it1.pop();
+          }
+          // Union order: the smaller head; a head equal to it advances.
+          auto union_pop = [&]() -> int {
+            const int jj = h0 < 0 ? h1 : (h1 < 0 ? h0 : min(h0, h1));
+            if (jj >= 0) {
+              if (h0 == jj) h0 = it0.pop();
+              if (h1 == jj) h1 = it1.pop();
+            }
+            return jj;
+          };
+          for (int j = SPARSE ? union_pop() : 0; SPARSE ? j >= 0 : j < nkv;
+               j = SPARSE ? union_pop() : j + 1, ++g) {
             const int s = g % C::kStages;
             const uint32_t ph = ((g / C::kStages) - 1) & 1;
             if (g >= C::kStages &&
@@ -576,8 +598,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               pm.w1 = words + kMaskWords;
             }
             if (!(ok = mbar_wait(&bars->q_full, units & 1, ab, status, timeout_ns))) break;
-            // Per-tile state, kept in scalars (t is a compile-time constant below).
-            int cur0 = pm.next(0, -1), cur1 = pm.next(1, -1);  // each tile's next key tile
+            // Per-tile state, kept in scalars (t is a compile-time constant below).  For each
+            // tile: cur_t = its next key tile, nx_t = the one after, nx2_t = the one after
+            // that (from a bit iterator over its mask words).
+            BitIter it0, it1;
+            it0.init(pm.w0);
+            it1.init(pm.w1);
+            int cur0 = it0.pop(), cur1 = it1.pop();
+            int nx0 = cur0 < 0 ? -1 : it0.pop(), nx1 = cur1 < 0 ? -1 : it1.pop();
+            int nx20 = nx0 < 0 ? -1 : it0.pop(), nx21 = nx1 < 0 ? -1 : it1.pop();
             bool sd0 = false, sd1 = false;                      // S_t(cur_t) issued
             bool fp0 = true, fp1 = true;                        // first PV of the unit
             bool ls0 = cur0 < 0, ls1 = cur1 < 0;                // no S left to issue for t
@@ -590,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             if (cur0 < 0) umma_commit(&bars->o_done[0]);  // nothing accumulated: done
             if (cur1 < 0) umma_commit(&bars->o_done[1]);
-            int j = pm.next_any(-1);
+            int j = cur0 < 0 ? cur1 : (cur1 < 0 ? cur0 : min(cur0, cur1));
             int gu = g;  // ring position of key tile j
             if (j >= 0) {
               const int s = gu % C::kStages;
@@ -601,12 +630,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (cur0 == j) {
                 issue_s(0, s);
                 sd0 = true;
-                ls0 = pm.next(0, j) < 0;
+                ls0 = nx0 < 0;
               }
               if (cur1 == j) {
                 issue_s(1, s);
                 sd1 = true;
-                ls1 = pm.next(1, j) < 0;
+                ls1 = nx1 < 0;
               }
               umma_commit(&bars->k_empty[s]);  // every tile active at j is served
             }
@@ -616,11 +645,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int sn = (gu + 1) % C::kStages;
               // Everything this step needs from the masks, before any wait.
               const bool on0 = cur0 == j, on1 = cur1 == j;
-              const int nt0 = on0 ? pm.next(0, j) : cur0;
-              const int nt1 = on1 ? pm.next(1, j) : cur1;
+              const int nt0 = on0 ? nx0 : cur0;
+              const int nt1 = on1 ? nx1 : cur1;
               const int jn = (nt0 < 0) ? nt1 : ((nt1 < 0) ? nt0 : min(nt0, nt1));
-              const bool last0 = nt0 < 0 || pm.next(0, nt0) < 0;
-              const bool last1 = nt1 < 0 || pm.next(1, nt1) < 0;
+              const bool last0 = nt0 < 0 || (on0 ? nx20 : nx0) < 0;
+              const bool last1 = nt1 < 0 || (on1 ? nx21 : nx1) < 0;
               // S owed on j (its K stage is still held for it).
               const bool owe0 = on0 && !sd0, owe1 = on1 && !sd1;
               if (owe0 || owe1) {
@@ -674,6 +703,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!(ok = pv_then_next_s(std::integral_constant<int, 1>{}, on1, fp1, cur1, sd1, ls1,
                                         nt1, last1, true)))
                 break;
+              // Advance the lookahead of the tiles that moved on.
+              if (on0) {
+                nx0 = nx20;
+                nx20 = nx20 < 0 ? -1 : it0.pop();
+              }
+              if (on1) {
+                nx1 = nx21;
+                nx21 = nx21 < 0 ? -1 : it1.pop();
+              }
               if (jn >= 0 && !((cur0 == jn && !sd0) || (cur1 == jn && !sd1)))
                 umma_commit(&bars->k_empty[sn]);  // no S owed on jn: its K stage is free
               release_q();
