@@ -37,6 +37,9 @@ METRIC = "attention fwd/bwd TFLOPS on 1 B200 vs BF16 tensor-core peak (fraction 
 UNIT = "TFLOPS"
 L2_BYTES = 126 * 2 ** 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# NVIDIA's dense (no 2:4 sparsity) BF16 tensor-core figure for one B200, as given in the
+# hardware notes this build was made with (the datasheet itself is not reachable offline).
+NOMINAL_DENSE_BF16_TFLOPS = 2250.0
 KERNELS_PER_STEP = 4  # fwd, bwd_pre, bwd_main, dq_convert
 
 
@@ -345,6 +348,7 @@ def run_ours(args, rank, world, local_rank):
                          "frac": round(main_tflops / peak_sus, 4),
                          "peak_kind": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
                          "frac_of_burst_peak": round(main_tflops / peak_burst, 4),
+                         "frac_of_nominal_dense_bf16": round(main_tflops / NOMINAL_DENSE_BF16_TFLOPS, 4),
                          "traffic": traffic},
             "clocks": clocks,
             "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
