@@ -583,6 +583,47 @@ int fa_debug_exp2(const float* x, float* y_poly, float* y_hw, int n, void* strea
   return from_cuda(fa::launch_debug_exp2(x, y_poly, y_hw, n, static_cast<cudaStream_t>(stream)));
 }
 
+int fa_debug_tma_tile(const void* x, void* y, int B, int N, int H, int d, int b, int h, int row0,
+                      int chunk, void* stream) {
+  if (!x || !y) return FA_ERR_INVALID_ARG;
+  int rc = check_shape(B, H, N, d, 1.0f);
+  if (rc) return rc;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (b < 0 || b >= B || h < 0 || h >= H || row0 < 0 || row0 >= N || chunk < 0 ||
+      chunk >= d / 64)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16)) return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  if ((rc = device_info(&di))) return rc;
+  CUtensorMap tm;
+  if ((rc = encode_bnhd(&tm, x, B, N, H, d))) return rc;
+  return from_cuda(fa::launch_debug_tma_tile(tm, y, b, h, row0, chunk, di.status,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+int fa_debug_tmem_roundtrip(const uint32_t* in, uint32_t* out, int ncols, void* stream) {
+  if (!in || !out) return FA_ERR_INVALID_ARG;
+  if (ncols != 32 && ncols != 64 && ncols != 128 && ncols != 256) return FA_ERR_UNSUPPORTED;
+  if (!aligned(in, 4) || !aligned(out, 4)) return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  return from_cuda(fa::launch_debug_tmem_roundtrip(in, out, ncols, static_cast<cudaStream_t>(stream)));
+}
+
+int fa_debug_fwd_schedule(int B, int H, int N, int causal, int grid, int* units, int max_rounds,
+                          void* stream) {
+  if (!units || B < 1 || H < 1 || N < 1 || grid < 1 || grid > 65535 || max_rounds < 1)
+    return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(grid) * max_rounds > (1LL << 28)) return FA_ERR_INVALID_ARG;
+  if (!aligned(units, 4)) return FA_ERR_MISALIGNED;
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  return from_cuda(fa::launch_debug_schedule(B, H, N, causal ? 1 : 0, grid, units, max_rounds,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
 int fa_debug_wait_timeout(long long timeout_ns, void* stream) {
   if (timeout_ns < 1000 || timeout_ns > 10000000000LL) return FA_ERR_INVALID_ARG;
   DeviceInfo di;

@@ -2,6 +2,8 @@
 //   * one 128 x n x k tcgen05.mma tile with operands written to shared memory in the
 //     128-byte-swizzled layouts the attention kernels use (K-major and MN-major), or with A
 //     staged in tensor memory as packed bf16 pairs;
+//   * one TMA box load through the kernels' tensor-map encoding, read back unswizzled;
+//   * a tensor-memory store / load round trip;
 //   * a bounded mbarrier wait that is made to run out, to exercise the timeout path.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -120,6 +122,80 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+// One 128-row x 64-element bf16 box of a [B][N][H][d] tensor through TMA (128-byte swizzle,
+// the attention kernels' encoding), copied out row-major (unswizzled) into y[128][64].
+__global__ void __launch_bounds__(128, 1)
+    tma_tile_kernel(const __grid_constant__ CUtensorMap tm, __nv_bfloat16* __restrict__ y, int b,
+                    int h, int row0, int chunk, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* tile = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(tile + 16384);
+  Abort* ab = reinterpret_cast<Abort*>(tile + 16384 + 64);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    ab->flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bar, 16384);
+    tma_load_4d(tile, &tm, bar, chunk * 64, h, row0, b, policy_evict_first());
+  }
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, 0, ab, status, kDefaultWaitTimeoutNs));
+  if (ok) {
+    const int r = threadIdx.x;
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      reinterpret_cast<uint4*>(y + r * 64)[c] =
+          *reinterpret_cast<const uint4*>(tile + sw128_offset(r, c));
+  }
+}
+
+// Lane r writes in[r][0..ncols) into tensor-memory columns [0, ncols) with tcgen05.st and
+// reads them back with tcgen05.ld into out[r][0..ncols).
+__global__ void __launch_bounds__(128, 1)
+    tmem_roundtrip_kernel(const uint32_t* __restrict__ in, uint32_t* __restrict__ out, int ncols) {
+  __shared__ uint32_t tslot;
+  const int warp = threadIdx.x >> 5;
+  if (warp == 0) {
+    tmem_alloc(&tslot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t lane_base = tslot + (static_cast<uint32_t>(warp * 32) << 16);
+  const int r = threadIdx.x;
+  for (int c0 = 0; c0 < ncols; c0 += 32) {
+    uint32_t v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = in[r * ncols + c0 + i];
+    tmem_st32(lane_base + c0, v);
+  }
+  tmem_st_wait();
+  for (int c0 = 0; c0 < ncols; c0 += 64) {
+    if (c0 + 64 <= ncols) {
+      uint32_t v[64];
+      tmem_ld64(lane_base + c0, v);
+#pragma unroll
+      for (int i = 0; i < 64; ++i) out[r * ncols + c0 + i] = v[i];
+    } else {
+      uint32_t v[32];
+      tmem_ld32(lane_base + c0, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) out[r * ncols + c0 + i] = v[i];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) {
+    __syncwarp();
+    tmem_dealloc(tslot, 256);
+  }
+}
+
 __global__ void wait_timeout_kernel(uint64_t timeout_ns, int* status) {
   __shared__ uint64_t bar;
   __shared__ Abort ab;
@@ -166,6 +242,23 @@ cudaError_t launch_debug_umma(const void* a, const void* b, float* c, int n, int
   dbg::umma_tile_kernel<<<1, 128, smem, s>>>(static_cast<const __nv_bfloat16*>(a),
                                              static_cast<const __nv_bfloat16*>(b), c, n, k, mode,
                                              status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_tma_tile(const CUtensorMap& tm, void* y, int b, int h, int row0,
+                                  int chunk, int* status, cudaStream_t s) {
+  const int smem = 16384 + 256 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(dbg::tma_tile_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dbg::tma_tile_kernel<<<1, 128, smem, s>>>(tm, static_cast<__nv_bfloat16*>(y), b, h, row0,
+                                            chunk, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_tmem_roundtrip(const uint32_t* in, uint32_t* out, int ncols,
+                                        cudaStream_t s) {
+  dbg::tmem_roundtrip_kernel<<<1, 128, 0, s>>>(in, out, ncols);
   return cudaGetLastError();
 }
 

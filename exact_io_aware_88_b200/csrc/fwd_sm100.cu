@@ -909,6 +909,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Self-test: CTA c of a `grid`-CTA launch writes, round by round, the units the forward's
+// persistent schedule hands it (bh * num_pairs + pair), then -1.
+template <bool CAUSAL>
+__global__ void schedule_kernel(int BH, int num_pairs, int* __restrict__ out, int max_rounds) {
+  if (threadIdx.x != 0) return;
+  const int G = gridDim.x;
+  const int num_units = BH * num_pairs;
+  for (int r = 0; r < max_rounds; ++r) {
+    const int u = unit_of_round(r, G);
+    if (u >= num_units) {
+      out[blockIdx.x * max_rounds + r] = -1;
+      return;
+    }
+    const Unit x = decode_unit<CAUSAL>(u, BH, num_pairs);
+    out[blockIdx.x * max_rounds + r] = x.bh * num_pairs + x.pair;
+  }
+}
+
 template <int D, bool CAUSAL, bool F8 = false, bool SPARSE = false>
 static cudaError_t launch_t(const FwdArgs& a, cudaStream_t st) {
   using C = Cfg<D, F8>;
@@ -954,6 +972,16 @@ cudaError_t launch_fwd_block_sparse(const FwdArgs& a, cudaStream_t s) {
                     : fwd::launch_t<64, false, false, true>(a, s);
   return a.causal ? fwd::launch_t<128, true, false, true>(a, s)
                   : fwd::launch_t<128, false, false, true>(a, s);
+}
+
+cudaError_t launch_debug_schedule(int B, int H, int N, int causal, int grid, int* out,
+                                  int max_rounds, cudaStream_t s) {
+  const int num_pairs = (N + 2 * fwd::BM - 1) / (2 * fwd::BM);
+  if (causal)
+    fwd::schedule_kernel<true><<<grid, 32, 0, s>>>(B * H, num_pairs, out, max_rounds);
+  else
+    fwd::schedule_kernel<false><<<grid, 32, 0, s>>>(B * H, num_pairs, out, max_rounds);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_fwd_fp8(const FwdArgs& a, cudaStream_t s) {

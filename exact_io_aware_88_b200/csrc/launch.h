@@ -80,6 +80,12 @@ cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float
 cudaError_t launch_debug_umma(const void* a, const void* b, float* c, int n, int k, int mode,
                               int* status, cudaStream_t s);
 cudaError_t launch_debug_wait_timeout(uint64_t timeout_ns, int* status, cudaStream_t s);
+cudaError_t launch_debug_tma_tile(const CUtensorMap& tm, void* y, int b, int h, int row0,
+                                  int chunk, int* status, cudaStream_t s);
+cudaError_t launch_debug_tmem_roundtrip(const uint32_t* in, uint32_t* out, int ncols,
+                                        cudaStream_t s);
+cudaError_t launch_debug_schedule(int B, int H, int N, int causal, int grid, int* out,
+                                  int max_rounds, cudaStream_t s);
 cudaError_t launch_debug_exp2(const float* x, float* y_poly, float* y_hw, int n, cudaStream_t s);
 
 }  // namespace fa

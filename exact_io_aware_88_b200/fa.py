@@ -95,6 +95,12 @@ _lib.fa_debug_exp2.argtypes = [_P, _P, _P, _I, _P]
 _lib.fa_debug_exp2.restype = _I
 _lib.fa_debug_wait_timeout.argtypes = [ctypes.c_longlong, _P]
 _lib.fa_debug_wait_timeout.restype = _I
+_lib.fa_debug_tma_tile.argtypes = [_P, _P] + [_I] * 8 + [_P]
+_lib.fa_debug_tma_tile.restype = _I
+_lib.fa_debug_tmem_roundtrip.argtypes = [_P, _P, _I, _P]
+_lib.fa_debug_tmem_roundtrip.restype = _I
+_lib.fa_debug_fwd_schedule.argtypes = [_I] * 5 + [_P, _I, _P]
+_lib.fa_debug_fwd_schedule.restype = _I
 
 # Every symbol the C headers declare, for the ABI self-check.
 EXPORTED = sorted(["fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess", "fa_bwd_kv",
@@ -103,7 +109,8 @@ EXPORTED = sorted(["fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_determi
                    "fa_fp8_quantize_workspace_bytes", "fa_fp8_quantize", "fa_fwd_fp8",
                    "fa_fwd_block_sparse_workspace_bytes", "fa_read_device_status", "fa_status_string",
                    "fa_version", "fa_debug_umma_tile", "fa_debug_wait_timeout",
-                   "fa_debug_exp2"])
+                   "fa_debug_exp2", "fa_debug_tma_tile", "fa_debug_tmem_roundtrip",
+                   "fa_debug_fwd_schedule"])
 
 
 def _ptr(x) -> Optional[int]:
@@ -238,6 +245,19 @@ def fa_debug_umma_tile(a, b, c, n, k, mode, stream=None) -> int:
 
 def fa_debug_exp2(x, y_poly, y_hw, n, stream=None) -> int:
     return _lib.fa_debug_exp2(_ptr(x), _ptr(y_poly), _ptr(y_hw), int(n), _stream(stream))
+
+
+def fa_debug_tma_tile(x, y, B, N, H, d, b, h, row0, chunk, stream=None) -> int:
+    return _lib.fa_debug_tma_tile(_ptr(x), _ptr(y), B, N, H, d, b, h, row0, chunk, _stream(stream))
+
+
+def fa_debug_tmem_roundtrip(inp, out, ncols, stream=None) -> int:
+    return _lib.fa_debug_tmem_roundtrip(_ptr(inp), _ptr(out), int(ncols), _stream(stream))
+
+
+def fa_debug_fwd_schedule(B, H, N, causal, grid, units, max_rounds, stream=None) -> int:
+    return _lib.fa_debug_fwd_schedule(B, H, N, int(causal), grid, _ptr(units), max_rounds,
+                                      _stream(stream))
 
 
 def fa_debug_wait_timeout(timeout_ns, stream=None) -> int:

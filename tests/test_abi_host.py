@@ -130,6 +130,17 @@ def test_block_sparse_workspace_is_the_packed_mask(fa):
     assert call(A16, 1 << 20, N=131073) == fa.FA_ERR_UNSUPPORTED
 
 
+def test_primitive_self_tests_reject_bad_arguments(fa):
+    assert fa.fa_debug_tma_tile(A16, A16, 1, 300, 2, 96, 0, 0, 0, 0, stream=0) == fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_debug_tma_tile(A16, A16, 1, 300, 2, 64, 0, 0, 300, 0, stream=0) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_debug_tma_tile(A16, A16, 1, 300, 2, 64, 0, 0, 0, 1, stream=0) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_debug_tma_tile(A16 + 8, A16, 1, 300, 2, 64, 0, 0, 0, 0, stream=0) == fa.FA_ERR_MISALIGNED
+    assert fa.fa_debug_tmem_roundtrip(A16, A16, 48, stream=0) == fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_debug_tmem_roundtrip(None, A16, 64, stream=0) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_debug_fwd_schedule(1, 1, 128, 0, 0, A16, 4, stream=0) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_debug_fwd_schedule(1, 1, 128, 0, 4, A16 + 2, 4, stream=0) == fa.FA_ERR_MISALIGNED
+
+
 def test_debug_entry_points_reject_bad_arguments(fa):
     assert fa.fa_debug_umma_tile(A16, A16, A16, 96, 64, 0, stream=0) == fa.FA_ERR_UNSUPPORTED
     assert fa.fa_debug_umma_tile(A16, A16, A16, 64, 64, 3, stream=0) == fa.FA_ERR_UNSUPPORTED
