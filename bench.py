@@ -621,6 +621,36 @@ def run_sweep(path: str, reps: int = 20, warmup: int = 3):
         raise RuntimeError("device status word reports a timeout")
 
 
+KERNEL_CASES = ("fwd_d64_N4096", "fwd_fp8_N4096")
+
+
+def run_kernel_case(name: str, launches: int = 4):
+    """A few launches of one kernel on one workload, for a profiler to capture: the head-dim
+    64 forward (fwd_d64, N=4096, non-causal) or the E4M3 forward (N=4096, H=16, d=128,
+    non-causal, after one fa_fp8_quantize).  Prints one line; nothing is timed."""
+    import torch
+    from exact_io_aware_88_b200 import fa
+    if name == "fwd_d64_N4096":
+        w = synthetic.fwd_sweep(64, 4096, False)
+        t = synthetic.draw_workload(w)
+        q, k, v = (t[n].cuda() for n in ("q", "k", "v"))
+        for _ in range(launches):
+            fa.attention_forward(q, k, v, causal=False)
+    elif name == "fwd_fp8_N4096":
+        B, N, H, d = 4, 4096, 16, 128
+        t = synthetic.draw(B, N, H, d, 1006, "bf16")
+        q, k, v = (t[n].cuda() for n in ("q", "k", "v"))
+        q8, k8, vt8, sc = fa.fp8_quantize(q, k, v, synthetic.draw_signs(d, 1007).cuda())
+        for _ in range(launches):
+            fa.attention_forward_fp8(q8, k8, vt8, sc, causal=False)
+    else:
+        raise ValueError(f"unknown kernel case {name}")
+    torch.cuda.synchronize()
+    if fa.fa_read_device_status() != 0:
+        raise RuntimeError("device status word reports a timeout")
+    print(json.dumps({"kernel_case": name, "launches": launches}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -629,12 +659,17 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--N", type=int, default=16384, choices=[1024, 2048, 4096, 8192, 16384, 65536])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-case", choices=KERNEL_CASES, default=None,
+                    help="run a few launches of one kernel (for a profiler) and exit")
     ap.add_argument("--sweep", metavar="PATH", default=None,
                     help="time every workload of the benchmark sweep into PATH (JSON lines) "
                          "instead of the single-step measurement")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.kernel_case:
+        run_kernel_case(args.kernel_case)
+        return 0
     if args.sweep:
         run_sweep(args.sweep)
         return
