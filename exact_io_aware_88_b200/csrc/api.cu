@@ -16,7 +16,8 @@
 
 namespace {
 
-// Library-owned device status word (FA_OK / FA_ERR_TIMEOUT); one per device context.
+// Library-owned device status word (FA_OK / FA_ERR_TIMEOUT / FA_ERR_INTERNAL); one per
+// device context.
 __device__ int g_fa_status = 0;
 
 constexpr int kMaxDevices = 64;
@@ -162,6 +163,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_WORKSPACE: return "workspace missing or too small";
     case FA_ERR_CUDA: return "CUDA error";
     case FA_ERR_TIMEOUT: return "device-side wait timed out";
+    case FA_ERR_INTERNAL: return "internal consistency check failed (library defect)";
     default: return "unknown status";
   }
 }

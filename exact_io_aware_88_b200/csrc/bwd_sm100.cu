@@ -87,6 +87,9 @@ struct Bars {
   uint64_t s_full, dp_full, p_ready, ds_ready, dq_full, dq_empty, dkdv_done, drain;
   uint32_t tmem_base;
   Abort abort;
+  // End-of-CTA protocol check, each must equal the CTA's query-tile count: [0] Q tiles and
+  // [1] dO tiles loaded, [2] MMA steps, [3 + h] compute warpgroup h's steps, [5] dQ drains.
+  int count[6];
 };
 static_assert(sizeof(Bars) <= 256, "barrier block larger than its shared-memory region");
 
@@ -193,6 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t colS = C::kColS + 64 * half;
     const uint32_t colDP = C::kColDP + 64 * half;
     bool ok = true;
+    int steps_done = 0;
     for (int n = 0; n < nq; ++n) {
       const int i = i_begin + n;
       const int q0 = i * BN;
@@ -270,7 +274,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars->ds_ready);
+      ++steps_done;
     }
+    if ((warp & 3) == 0 && lane == 0) bars->count[3 + half] = steps_done;
     // ---------------------------------------------------------------- dK / dV epilogue
     // Warpgroup 0 writes dK, warpgroup 1 writes dV.
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->dkdv_done, 0, ab, status, timeout_ns));
@@ -304,7 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;  // query row within the tile
     const uint32_t lane_base = tbase + (static_cast<uint32_t>(quarter * 32) << 16);
-    for (int n = 0; WITH_DQ && n < nq; ++n) {
+    int drains = WITH_DQ ? 0 : nq;
+    for (int n = 0; WITH_DQ && n < nq; ++n, ++drains) {
       const int q = (i_begin + n) * BN + r;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_full, n & 1, ab, status, timeout_ns));
       if (!ok) break;
@@ -348,6 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if (warp == 8 && lane == 0) bars->count[5] = drains;
   } else {
     regs_set<kRegsLaunch, kRegsOther>();
     if (warp == kWarpLoad) {
@@ -388,6 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         c * 64, h, i * BN, b, pol_q);
           issued_do = n + 1;
         }
+        bars->count[0] = issued_q;
+        bars->count[1] = issued_do;
         // Drain every copy into shared memory before the CTA may exit.
         Abort local{0};
         mbar_wait(&bars->kv_full, 0, &local, status, timeout_ns);
@@ -447,6 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         bool ok = mbar_wait(&bars->kv_full, 0, ab, status, timeout_ns) && issue_s(0) && issue_dp(0);
+        int mma_steps = 0;
         for (int n = 0; ok && n < nq; ++n) {
           const int sq = n % C::kQStages, sd = n % C::kDOStages;
           const uint32_t qb = aQ + sq * C::kTileBytes, dob = aDO + sd * C::kTileBytes;
@@ -487,8 +498,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sdesc_sw128(qb + kk * 2048, C::kChunkBytes, 1024), id_dkdv, (n > 0 || kk > 0));
           }
           umma_commit(&bars->q_empty[sq]);
+          ++mma_steps;
           if (n + 1 < nq && !issue_dp(n + 1)) break;
         }
+        bars->count[2] = mma_steps;
         umma_commit(&bars->dkdv_done);
         umma_commit(&bars->drain);
         Abort local{0};
@@ -500,6 +513,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Every role must have done one step per query tile (skipped after a timed-out wait).
+  if (threadIdx.x == 0 && !*reinterpret_cast<volatile int*>(&ab->flag)) {
+    bool agree = true;
+#pragma unroll
+    for (int i = 0; i < 6; ++i) agree = agree && bars->count[i] == nq;
+    if (!agree) atomicCAS(status, FA_OK, FA_ERR_INTERNAL);
+  }
   if (warp == kWarpMma) {
     __syncwarp();
     tmem_dealloc(tbase, kTmemCols);

@@ -97,6 +97,10 @@ struct Bars {
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint64_t s_full[2], p_full[2], o_done[2], o_free[2];
   uint64_t p_half[2];  // P_t of the first 64 keys is in TMEM (and O_t rescaled)
+  // End-of-CTA protocol check: [0] K/V tiles loaded, [1] units loaded, [2] K/V tiles
+  // consumed by the MMA lane, [3] its units, [4 + t] softmax t's steps, [6 + t] S products
+  // issued for tile t, [8 + t] softmax t's units.
+  int count[10];
   uint64_t drain;
   uint32_t tmem_base;
   Abort abort;
@@ -535,6 +539,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             empty ? -INFINITY : (m + __log2f(l)) * 0.69314718055994531f;
       }
     }
+    if ((warp & 3) == 0 && lane == 0) {
+      bars->count[4 + t] = ns;
+      bars->count[8 + t] = units;
+    }
   } else {
     regs_set<kRegsLaunch, kRegsOther<F8>>();
     if (warp == kWarpLoad) {
@@ -617,6 +625,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Drain: no copy into shared memory may still be in flight when the CTA exits.
         // Only the last Q pair and the last kStages K/V tiles can be outstanding.  (On the
         // abort path a V copy may not have been issued; its wait then runs out harmlessly.)
+        bars->count[0] = g;
+        bars->count[1] = units;
         Abort local{0};
         if (units > 0) mbar_wait(&bars->q_full, (units - 1) & 1, &local, status, timeout_ns);
         for (int gg = max(0, g - C::kStages); gg < g; ++gg) {
@@ -638,7 +648,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         int units = 0;        // units finished
         int np[2] = {0, 0};   // p_full phases consumed per tile
         bool ok = true;
+        int s_issued0 = 0, s_issued1 = 0;  // S products issued per tile (protocol check)
         auto issue_s = [&](int t, int s) {  // S_t = Q_t K^T (both K-major over the head dim)
+          (t ? s_issued1 : s_issued0) += 1;
           const uint32_t kb = aK + s * C::kTileBytes;
           const uint32_t qb = aQ + t * C::kTileBytes;
           // One MMA per 32 bytes of the head dim (16 bf16 or 32 E4M3 elements).
@@ -892,6 +904,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++units;
           }
         }
+        bars->count[2] = g;
+        bars->count[3] = units;
+        bars->count[6] = s_issued0;
+        bars->count[7] = s_issued1;
         // Drain every MMA this thread issued before TMEM is released.
         umma_commit(&bars->drain);
         Abort local{0};
@@ -903,6 +919,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // The roles must agree on what they did (skipped after a timed-out wait, when they may
+  // not): every K/V tile loaded was consumed, every unit was seen by all four roles, and
+  // each softmax warpgroup took exactly one step per S product of its tile.
+  if (threadIdx.x == 0 && !*reinterpret_cast<volatile int*>(&ab->flag)) {
+    const int* c = bars->count;
+    const bool agree = c[0] == c[2] && c[1] == c[3] && c[3] == c[8] && c[3] == c[9] &&
+                       c[4] == c[6] && c[5] == c[7];
+    if (!agree) atomicCAS(status, FA_OK, FA_ERR_INTERNAL);
+  }
   if (warp == kWarpMma) {
     __syncwarp();
     tmem_dealloc(tbase, kTmemCols);

@@ -27,6 +27,7 @@ FA_ERR_MISALIGNED = 3
 FA_ERR_WORKSPACE = 4
 FA_ERR_CUDA = 5
 FA_ERR_TIMEOUT = 6
+FA_ERR_INTERNAL = 7
 FA_DTYPE_BF16 = 0
 FA_DTYPE_FP16 = 1
 

@@ -30,7 +30,11 @@
  *    nothing was launched and no output was touched.  No C++ exception crosses the ABI.
  *  - Device-side failures (a bounded wait inside a kernel that ran out) do not trap the
  *    GPU: the kernel records FA_ERR_TIMEOUT in a library-owned device status word, tears
- *    its CTA down cleanly and returns; read it with fa_read_device_status().
+ *    its CTA down cleanly and returns; read it with fa_read_device_status().  At the end
+ *    of every CTA the main forward kernel (fa_fwd, fa_fwd_block_sparse, fa_fwd_fp8) and the
+ *    backward's key-tile kernel (fa_bwd, fa_bwd_kv) also check that their warp roles agree
+ *    on the work done (tiles loaded = consumed, steps per role) and record FA_ERR_INTERNAL
+ *    if not.
  */
 #ifndef FA_H_
 #define FA_H_
@@ -49,7 +53,9 @@ typedef enum {
   FA_ERR_MISALIGNED = 3,  /* a pointer not 16-byte aligned                                */
   FA_ERR_WORKSPACE = 4,   /* workspace null or smaller than fa_bwd_workspace_bytes()      */
   FA_ERR_CUDA = 5,        /* a CUDA runtime / driver call failed (launch, attribute, ...) */
-  FA_ERR_TIMEOUT = 6      /* a device-side bounded wait expired (read via status word)    */
+  FA_ERR_TIMEOUT = 6,     /* a device-side bounded wait expired (read via status word)    */
+  FA_ERR_INTERNAL = 7     /* a kernel's end-of-CTA protocol check failed: a library defect
+                             (read via status word; the results of that call are not valid) */
 } fa_status;
 
 /* Forward pass, bf16 in / bf16 out, fp32 accumulation and statistics.
@@ -210,8 +216,8 @@ int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* 
                int B, int H, int N, int d, int causal, float scale, void* stream);
 
 /* Synchronises `stream`, then returns and clears the library's device status word
- * (FA_OK or FA_ERR_TIMEOUT).  If `status_out` is non-null the raw word is also stored
- * there (host pointer).  Returns FA_ERR_CUDA if the synchronisation itself failed. */
+ * (FA_OK, FA_ERR_TIMEOUT or FA_ERR_INTERNAL; the first failure recorded wins).  If
+ * `status_out` is non-null the raw word is also stored there (host pointer).  Returns FA_ERR_CUDA if the synchronisation itself failed. */
 int fa_read_device_status(int* status_out, void* stream);
 
 /* Static, human-readable name of a status code. */
