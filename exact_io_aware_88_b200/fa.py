@@ -272,10 +272,34 @@ def _check(fn: str, rc: int):
         raise FAError(fn, rc)
 
 
-def _shape(q: torch.Tensor):
-    if q.dim() != 4:
+def _shape(q) -> Tuple[int, int, int, int]:
+    if not isinstance(q, torch.Tensor) or q.dim() != 4:
         raise ValueError("expected [B, N, H, d] tensors")
-    return q.shape
+    return tuple(q.shape)
+
+
+def _require(*specs) -> None:
+    """Each spec is (name, tensor, shape, dtypes).  Raises ValueError unless every tensor is
+    contiguous, exactly `shape`, one of `dtypes`, and on the same CUDA device as the first.
+    Shapes, dtypes and layouts are checked for all tensors before devices.  The kernels read
+    and write whole extents through raw pointers, so a tensor that fails any of these would
+    be read or written out of bounds."""
+    for name, t, shape, dtypes in specs:
+        if not isinstance(t, torch.Tensor):
+            raise ValueError(f"{name} must be a torch.Tensor")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+        if t.dtype not in dtypes:
+            raise ValueError(f"{name}: expected dtype {' or '.join(map(str, dtypes))}, "
+                             f"got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    dev = specs[0][1].device
+    for name, t, _, _ in specs:
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, expected {dev}")
 
 
 def attention_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
@@ -284,17 +308,21 @@ def attention_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal:
     """O, LSE for [B, N, H, d] CUDA tensors (bf16 -> fa_fwd, fp32 -> fa_fwd_f32)."""
     B, N, H, d = _shape(q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    for t in (q, k, v):
-        if not (t.is_cuda and t.is_contiguous() and t.shape == q.shape and t.dtype == q.dtype):
-            raise ValueError("q, k, v must be contiguous CUDA tensors of one shape and dtype")
-    o = torch.empty_like(q) if out is None else out
-    l = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
-    if q.dtype == torch.bfloat16:
-        _check("fa_fwd", fa_fwd(q, k, v, o, l, B, H, N, d, causal, scale))
-    elif q.dtype == torch.float32:
-        _check("fa_fwd_f32", fa_fwd_f32(q, k, v, o, l, B, H, N, d, causal, scale))
-    else:
-        raise ValueError(f"unsupported dtype {q.dtype}")
+    x = (B, N, H, d)
+    specs = [("q", q, x, (torch.bfloat16, torch.float32)), ("k", k, x, (q.dtype,)),
+             ("v", v, x, (q.dtype,))]
+    if out is not None:
+        specs.append(("out", out, x, (q.dtype,)))
+    if lse is not None:
+        specs.append(("lse", lse, (B, H, N), (torch.float32,)))
+    _require(*specs)
+    with torch.cuda.device(q.device):
+        o = torch.empty_like(q) if out is None else out
+        l = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+        if q.dtype == torch.bfloat16:
+            _check("fa_fwd", fa_fwd(q, k, v, o, l, B, H, N, d, causal, scale))
+        else:
+            _check("fa_fwd_f32", fa_fwd_f32(q, k, v, o, l, B, H, N, d, causal, scale))
     return o, l
 
 
@@ -303,13 +331,21 @@ def attention_backward(q, k, v, o, lse, dO, causal: bool = False, scale: Optiona
     """dQ, dK, dV for bf16 [B, N, H, d] CUDA tensors (fa_bwd, or fa_bwd_deterministic)."""
     B, N, H, d = _shape(q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
+    x, bf = (B, N, H, d), (torch.bfloat16,)
+    specs = [("q", q, x, bf), ("k", k, x, bf), ("v", v, x, bf), ("o", o, x, bf),
+             ("lse", lse, (B, H, N), (torch.float32,)), ("dO", dO, x, bf)]
+    if workspace is not None:
+        specs.append(("workspace", workspace, tuple(getattr(workspace, "shape", ())),
+                      (getattr(workspace, "dtype", None),)))
+    _require(*specs)
     nbytes = fa_bwd_workspace_bytes(B, H, N, d)
-    if workspace is None:
-        workspace = torch.empty(nbytes, device=q.device, dtype=torch.uint8)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    fn = fa_bwd_deterministic if deterministic else fa_bwd
-    _check(fn.__name__, fn(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale,
-                           workspace, workspace.numel() * workspace.element_size()))
+    with torch.cuda.device(q.device):
+        if workspace is None:
+            workspace = torch.empty(nbytes, device=q.device, dtype=torch.uint8)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        fn = fa_bwd_deterministic if deterministic else fa_bwd
+        _check(fn.__name__, fn(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale,
+                               workspace, workspace.numel() * workspace.element_size()))
     return dq, dk, dv
 
 
@@ -317,32 +353,45 @@ def attention_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: 
                      scale: Optional[float] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """O, LSE for q [B, Nq, H, d] against k, v [B, Nk, H, d] (bf16 or fp16), split-KV."""
     B, Nq, H, d = _shape(q)
-    Nk = k.shape[1]
+    Nk = _shape(k)[1]
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     dt = {torch.bfloat16: FA_DTYPE_BF16, torch.float16: FA_DTYPE_FP16}.get(q.dtype)
     if dt is None:
         raise ValueError(f"unsupported dtype {q.dtype}")
-    o = torch.empty_like(q)
-    lse = torch.empty((B, H, Nq), device=q.device, dtype=torch.float32)
-    nb = fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d)
-    ws = torch.empty(max(nb, 256), device=q.device, dtype=torch.uint8)
-    _check("fa_fwd_splitkv", fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, dt,
-                                            ws, ws.numel()))
+    _require(("q", q, (B, Nq, H, d), (q.dtype,)), ("k", k, (B, Nk, H, d), (q.dtype,)),
+             ("v", v, (B, Nk, H, d), (q.dtype,)))
+    with torch.cuda.device(q.device):
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, Nq), device=q.device, dtype=torch.float32)
+        nb = fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d)
+        ws = torch.empty(max(nb, 256), device=q.device, dtype=torch.uint8)
+        _check("fa_fwd_splitkv", fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale,
+                                                dt, ws, ws.numel()))
     return o, lse
 
 
 def attention_block_sparse(q, k, v, block_mask: torch.Tensor, causal: bool = False,
                            scale: Optional[float] = None):
-    """O, LSE for bf16 [B, N, H, d] tensors with a [ceil(N/128), ceil(N/128)] uint8 mask."""
+    """O, LSE for bf16 [B, N, H, d] tensors with a [ceil(N/128), ceil(N/128)] mask (nonzero =
+    block active; any integer or bool dtype, on any device)."""
     B, N, H, d = _shape(q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    m = block_mask.to(device=q.device, dtype=torch.uint8).contiguous()
-    o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
-    nb = fa_fwd_block_sparse_workspace_bytes(B, H, N, d)
-    ws = torch.empty(max(nb, 256), device=q.device, dtype=torch.uint8)
-    _check("fa_fwd_block_sparse", fa_fwd_block_sparse(q, k, v, o, lse, B, H, N, d, causal, scale,
-                                                      m, ws, ws.numel()))
+    nt = (N + 127) // 128
+    if not isinstance(block_mask, torch.Tensor) or tuple(block_mask.shape) != (nt, nt):
+        got = tuple(block_mask.shape) if isinstance(block_mask, torch.Tensor) else type(block_mask)
+        raise ValueError(f"block_mask: expected shape {(nt, nt)}, got {got}")
+    if block_mask.is_floating_point() or block_mask.is_complex():
+        raise ValueError(f"block_mask: expected an integer or bool dtype, got {block_mask.dtype}")
+    x, bf = (B, N, H, d), (torch.bfloat16,)
+    _require(("q", q, x, bf), ("k", k, x, bf), ("v", v, x, bf))
+    with torch.cuda.device(q.device):
+        m = (block_mask != 0).to(device=q.device, dtype=torch.uint8).contiguous()
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+        nb = fa_fwd_block_sparse_workspace_bytes(B, H, N, d)
+        ws = torch.empty(max(nb, 256), device=q.device, dtype=torch.uint8)
+        _check("fa_fwd_block_sparse", fa_fwd_block_sparse(q, k, v, o, lse, B, H, N, d, causal,
+                                                          scale, m, ws, ws.numel()))
     return o, lse
 
 
@@ -352,26 +401,37 @@ def fp8_quantize(q, k, v, signs: Optional[torch.Tensor]):
     (q8, k8, vt8, scales) as uint8 [B, N, H, d], uint8 [B, N, H, d], uint8 [B, H, d, Npad]
     and fp32 [3, B*H]."""
     B, N, H, d = _shape(q)
+    if signs is not None and (not isinstance(signs, torch.Tensor) or tuple(signs.shape) != (d,)):
+        got = tuple(signs.shape) if isinstance(signs, torch.Tensor) else type(signs)
+        raise ValueError(f"signs: expected shape {(d,)}, got {got}")
+    x, bf = (B, N, H, d), (torch.bfloat16,)
+    _require(("q", q, x, bf), ("k", k, x, bf), ("v", v, x, bf))
     npad = (N + 15) // 16 * 16
     dev = q.device
-    q8 = torch.empty((B, N, H, d), device=dev, dtype=torch.uint8)
-    k8 = torch.empty_like(q8)
-    vt8 = torch.empty((B, H, d, npad), device=dev, dtype=torch.uint8)
-    scales = torch.empty((3, B * H), device=dev, dtype=torch.float32)
-    nb = fa_fp8_quantize_workspace_bytes(B, H)
-    ws = torch.empty(max(nb, 256), device=dev, dtype=torch.uint8)
-    sg = None if signs is None else signs.to(device=dev, dtype=torch.float32).contiguous()
-    _check("fa_fp8_quantize", fa_fp8_quantize(q, k, v, sg, q8, k8, vt8, scales, B, H, N, d, ws,
-                                              ws.numel()))
+    with torch.cuda.device(dev):
+        q8 = torch.empty((B, N, H, d), device=dev, dtype=torch.uint8)
+        k8 = torch.empty_like(q8)
+        vt8 = torch.empty((B, H, d, npad), device=dev, dtype=torch.uint8)
+        scales = torch.empty((3, B * H), device=dev, dtype=torch.float32)
+        nb = fa_fp8_quantize_workspace_bytes(B, H)
+        ws = torch.empty(max(nb, 256), device=dev, dtype=torch.uint8)
+        sg = None if signs is None else signs.to(device=dev, dtype=torch.float32).contiguous()
+        _check("fa_fp8_quantize", fa_fp8_quantize(q, k, v, sg, q8, k8, vt8, scales, B, H, N, d,
+                                                  ws, ws.numel()))
     return q8, k8, vt8, scales
 
 
 def attention_forward_fp8(q8, k8, vt8, scales, causal: bool = False,
                           scale: Optional[float] = None):
     """O (bf16 [B, N, H, d]) and LSE (fp32 [B, H, N]) from fp8_quantize's operands."""
-    B, N, H, d = q8.shape
+    B, N, H, d = _shape(q8)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    o = torch.empty((B, N, H, d), device=q8.device, dtype=torch.bfloat16)
-    lse = torch.empty((B, H, N), device=q8.device, dtype=torch.float32)
-    _check("fa_fwd_fp8", fa_fwd_fp8(q8, k8, vt8, scales, o, lse, B, H, N, d, causal, scale))
+    npad = (N + 15) // 16 * 16
+    u8 = (torch.uint8,)
+    _require(("q8", q8, (B, N, H, d), u8), ("k8", k8, (B, N, H, d), u8),
+             ("vt8", vt8, (B, H, d, npad), u8), ("scales", scales, (3, B * H), (torch.float32,)))
+    with torch.cuda.device(q8.device):
+        o = torch.empty((B, N, H, d), device=q8.device, dtype=torch.bfloat16)
+        lse = torch.empty((B, H, N), device=q8.device, dtype=torch.float32)
+        _check("fa_fwd_fp8", fa_fwd_fp8(q8, k8, vt8, scales, o, lse, B, H, N, d, causal, scale))
     return o, lse
