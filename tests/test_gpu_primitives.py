@@ -3,7 +3,6 @@ a TMA box load through the attention kernels' tensor-map encoding, a tensor-memo
 store / load round trip, and the forward kernel's persistent schedule against a Python
 model of it.  Plus the memory claim of the source pages: the forward and backward need
 O(N d) device memory, never the N x N score matrix."""
-import numpy as np
 import pytest
 import torch
 
