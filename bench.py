@@ -475,11 +475,15 @@ def run_sweep(path: str, reps: int = 20, warmup: int = 3):
             assert fwd() == 0
             med, best = timed(fwd)
             elem = 4 if w.dtype == "f32" else 2
+            # Roofline time: the slower of the tensor-core time at the burst peak and the
+            # HBM time of the algorithmic bytes (read Q, K, V, write O and the LSE).
             hbm_floor = (4 * B * N * H * d * elem + 4 * B * H * N) / (hbm * 1e9) * 1e3  # ms
+            roof = max(w.fwd_flops() / (burst * 1e12) * 1e3, hbm_floor)
             rec = {"workload": w.label(), "pass": "fwd", "ms": round(med, 4), "ms_best": round(best, 4),
                    "tflops": round(w.fwd_flops() / (med * 1e-3) / 1e12, 1),
                    "frac_of_burst_peak": round(w.fwd_flops() / (med * 1e-3) / 1e12 / burst, 4),
-                   "hbm_floor_ms": round(hbm_floor, 4), "peak_source": peak_src}
+                   "hbm_floor_ms": round(hbm_floor, 4), "roofline_ms": round(roof, 4),
+                   "frac_of_roofline": round(roof / med, 4), "peak_source": peak_src}
             out.write(json.dumps(rec) + "\n")
             print(json.dumps(rec), file=sys.stderr)
             if w.backward:
@@ -491,11 +495,15 @@ def run_sweep(path: str, reps: int = 20, warmup: int = 3):
                                         w.scale, ws, nb, stream)
                 assert bwd() == 0
                 med, best = timed(bwd)
+                # Algorithmic bytes: read Q, K, V, O, dO and the LSE, write dQ, dK, dV.
+                bwd_floor = (8 * B * N * H * d * elem + 4 * B * H * N) / (hbm * 1e9) * 1e3
+                roof = max(w.bwd_flops() / (burst * 1e12) * 1e3, bwd_floor)
                 rec = {"workload": w.label(), "pass": "bwd", "ms": round(med, 4),
                        "ms_best": round(best, 4),
                        "tflops": round(w.bwd_flops() / (med * 1e-3) / 1e12, 1),
                        "frac_of_burst_peak": round(w.bwd_flops() / (med * 1e-3) / 1e12 / burst, 4),
-                       "peak_source": peak_src}
+                       "hbm_floor_ms": round(bwd_floor, 4), "roofline_ms": round(roof, 4),
+                       "frac_of_roofline": round(roof / med, 4), "peak_source": peak_src}
                 out.write(json.dumps(rec) + "\n")
                 print(json.dumps(rec), file=sys.stderr)
                 det = lambda: fa.fa_bwd_deterministic(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d,
