@@ -160,3 +160,30 @@ def test_incoherent_processing_lowers_fp8_attention_error():
             e.append(np.sqrt(np.mean((O - Or) ** 2)))
         err[name] = float(np.mean(e))
     assert err["plain"] / err["hadamard"] > 1.25, err
+
+
+def test_lossless_operands_give_exact_attention():
+    """Inputs whose values are exact in E4M3 after the per-head power-of-two scaling are
+    quantised without loss, so attention on the dequantised codes must equal exact attention
+    on the inputs.  Here Q takes values in {0, +-0.5, +-1, +-1.5, +-2} (max 2, scale 2^-7),
+    K the same times 4 (scale 2^-5) and V times 1/4 (scale 2^-9): each maps to E4M3 numbers
+    exactly, and the three scales differ, so this pins the scale bookkeeping (s_q, s_k, s_v),
+    the transposed V layout and the decoding together."""
+    rng = np.random.default_rng(21)
+    B, N, H, d = 1, 150, 2, 64
+    vals = np.array([0.0, 0.5, -0.5, 1.0, -1.0, 1.5, -1.5, 2.0, -2.0])
+    q, k, v = (vals[rng.integers(0, len(vals), size=(B, N, H, d))] for _ in range(3))
+    for x in (q, k, v):
+        x[0, 0, :, 0] = 2.0  # every head's max |x| is 2 before the factors below
+    k, v = 4.0 * k, 0.25 * v
+    r = fp8.quantize(q, k, v, None)
+    assert np.all(r["scales"][0] == 2.0 ** -7) and np.all(r["scales"][1] == 2.0 ** -5)
+    assert np.all(r["scales"][2] == 2.0 ** -9)
+    scale = 1.0 / math.sqrt(d)
+    for h in range(H):
+        for causal in (False, True):
+            O, L = fp8.attention_head(r["q8"][0, :, h], r["k8"][0, :, h], r["vt8"][0, h],
+                                      *r["scales"][:, h], scale, causal)
+            Or, Lr = oracle.forward_head(q[0, :, h], k[0, :, h], v[0, :, h], scale, causal)
+            np.testing.assert_allclose(O, Or, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(L, Lr, rtol=0, atol=1e-12)
