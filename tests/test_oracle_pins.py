@@ -92,7 +92,7 @@ def test_probability_rows_sum_to_one(causal):
     N, d = 20, 6
     Q, K = rnd(13, N, d), rnd(14, N, d)
     O, _ = forward_head(Q, K, np.eye(N), 0.5, causal)
-    np.testing.assert_allclose(O.sum(axis=1), 1.0, atol=1e-12)
+    np.testing.assert_allclose(O.sum(axis=1), 1.0, rtol=0, atol=1e-12)
     assert (O >= 0).all()
     if causal:
         assert np.all(np.triu(O, 1) == 0.0)
@@ -118,8 +118,8 @@ def test_noncausal_joint_permutation_of_keys_and_values():
     perm = np.random.default_rng(22).permutation(N)
     O0, l0 = forward_head(Q, K, V, 0.4, False)
     O1, l1 = forward_head(Q, K[perm], V[perm], 0.4, False)
-    np.testing.assert_allclose(O1, O0, atol=1e-13)
-    np.testing.assert_allclose(l1, l0, atol=1e-13)
+    np.testing.assert_allclose(O1, O0, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l1, l0, rtol=0, atol=1e-13)
 
 
 def test_causal_row_equals_noncausal_attention_over_its_prefix():
@@ -128,7 +128,7 @@ def test_causal_row_equals_noncausal_attention_over_its_prefix():
     Oc, lc = forward_head(Q, K, V, 0.6, True)
     for i in (0, 5, 16):
         Op, lp = forward_head(Q[i:i + 1], K[:i + 1], V[:i + 1], 0.6, False)
-        np.testing.assert_allclose(Oc[i], Op[0], atol=1e-14)
+        np.testing.assert_allclose(Oc[i], Op[0], rtol=0, atol=1e-14)
         assert abs(lc[i] - lp[0]) < 1e-14
 
 
@@ -138,9 +138,9 @@ def test_gradient_sum_rules(causal):
     Q, K, V, dO = (rnd(s, N, d) for s in (26, 27, 28, 29))
     dQ, dK, dV = backward_head(Q, K, V, dO, 0.35, causal)
     # each row of P sums to one:  sum_j dV_j = sum_i dO_i
-    np.testing.assert_allclose(dV.sum(axis=0), dO.sum(axis=0), atol=1e-12)
+    np.testing.assert_allclose(dV.sum(axis=0), dO.sum(axis=0), rtol=0, atol=1e-12)
     # each row of dS sums to zero:  sum_j dK_j = 0
-    np.testing.assert_allclose(dK.sum(axis=0), 0.0, atol=1e-12)
+    np.testing.assert_allclose(dK.sum(axis=0), 0.0, rtol=0, atol=1e-12)
 
 
 # ---------------------------------------------------------------- online softmax claim
@@ -181,8 +181,8 @@ def test_online_softmax_equals_whole_row_softmax(causal):
     Q, K, V = rnd(30, N, d), rnd(31, N, d), rnd(32, N, d)
     O, lse = forward_head(Q, K, V, 0.25, causal)
     Ot, lt = _blockwise_rescaled(Q, K, V, 0.25, causal, 16)
-    np.testing.assert_allclose(Ot, O, atol=1e-13)
-    np.testing.assert_allclose(lt, lse, atol=1e-13)
+    np.testing.assert_allclose(Ot, O, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lt, lse, rtol=0, atol=1e-13)
     if not causal:
         assert np.abs(_blockwise_naive(Q, K, V, 0.25, 16) - O).max() > 1e-2
 
@@ -220,7 +220,7 @@ def test_scalar_loop_twin_agrees(causal):
     dQ, dK, dV = backward_head(Q, K, V, dO, 0.9, causal)
     Os, ls, dQs, dKs, dVs = scalar_loop_head(Q.tolist(), K.tolist(), V.tolist(), dO.tolist(), 0.9, causal)
     for a, b in ((O, Os), (lse, ls), (dQ, dQs), (dK, dKs), (dV, dVs)):
-        np.testing.assert_allclose(a, np.array(b), atol=1e-13)
+        np.testing.assert_allclose(a, np.array(b), rtol=0, atol=1e-13)
 
 
 @pytest.mark.parametrize("causal", [False, True])
@@ -234,15 +234,15 @@ def test_matches_torch_sdpa_fp64_with_autograd(B, N, H, d, causal):
     out.backward(dO.transpose(1, 2))
     O, lse = oracle.forward(q.numpy(), k.numpy(), v.numpy(), scale, causal)
     dQ, dK, dV = oracle.backward(q.numpy(), k.numpy(), v.numpy(), dO.numpy(), scale, causal)
-    np.testing.assert_allclose(O, out.detach().transpose(1, 2).numpy(), atol=1e-12)
-    np.testing.assert_allclose(dQ, qt.grad.transpose(1, 2).numpy(), atol=1e-12)
-    np.testing.assert_allclose(dK, kt.grad.transpose(1, 2).numpy(), atol=1e-12)
-    np.testing.assert_allclose(dV, vt.grad.transpose(1, 2).numpy(), atol=1e-12)
+    np.testing.assert_allclose(O, out.detach().transpose(1, 2).numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dQ, qt.grad.transpose(1, 2).numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dK, kt.grad.transpose(1, 2).numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dV, vt.grad.transpose(1, 2).numpy(), rtol=0, atol=1e-12)
     # LSE against torch.logsumexp of the explicitly masked logits
     S = scale * torch.einsum("bihd,bjhd->bhij", q, k)
     if causal:
         S = S.masked_fill(torch.ones(N, N, dtype=torch.bool).triu(1), float("-inf"))
-    np.testing.assert_allclose(lse, torch.logsumexp(S, dim=-1).numpy(), atol=1e-12)
+    np.testing.assert_allclose(lse, torch.logsumexp(S, dim=-1).numpy(), rtol=0, atol=1e-12)
 
 
 # ---------------------------------------------------------------- sampled-row helpers
@@ -255,13 +255,13 @@ def test_row_sampled_helpers_match_whole_head():
         O, lse = forward_head(Q, K, V, scale, causal, slab=64)
         dQ, dK, dV = backward_head(Q, K, V, dO, scale, causal, slab=64)
         Or, lr = oracle.forward_rows(Q, K, V, scale, causal, rows)
-        np.testing.assert_allclose(Or, O[rows], atol=1e-13)
-        np.testing.assert_allclose(lr, lse[rows], atol=1e-13)
-        np.testing.assert_allclose(oracle.dq_rows(Q, K, V, dO, scale, causal, rows), dQ[rows], atol=1e-12)
+        np.testing.assert_allclose(Or, O[rows], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lr, lse[rows], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(oracle.dq_rows(Q, K, V, dO, scale, causal, rows), dQ[rows], rtol=0, atol=1e-12)
     dQ, dK, dV = backward_head(Q, K, V, dO, scale, True)
     tk, tv = oracle.kv_grad_tail(Q, K, V, dO, scale, 250)
-    np.testing.assert_allclose(tk, dK[250:], atol=1e-12)
-    np.testing.assert_allclose(tv, dV[250:], atol=1e-12)
+    np.testing.assert_allclose(tk, dK[250:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(tv, dV[250:], rtol=0, atol=1e-12)
 
 
 def test_slab_size_does_not_change_results():
@@ -270,11 +270,11 @@ def test_slab_size_does_not_change_results():
     for causal in (False, True):
         a = forward_head(Q, K, V, 0.5, causal, slab=N)
         b = forward_head(Q, K, V, 0.5, causal, slab=7)
-        np.testing.assert_allclose(a[0], b[0], atol=1e-14)
+        np.testing.assert_allclose(a[0], b[0], rtol=0, atol=1e-14)
         ga = backward_head(Q, K, V, dO, 0.5, causal, slab=N)
         gb = backward_head(Q, K, V, dO, 0.5, causal, slab=7)
         for x, y in zip(ga, gb):
-            np.testing.assert_allclose(x, y, atol=1e-12)
+            np.testing.assert_allclose(x, y, rtol=0, atol=1e-12)
 
 
 # ---------------------------------------------------------------- fewer queries than keys
@@ -286,8 +286,8 @@ def test_single_last_query_sees_every_key():
     Q, K, V = rnd(90, 1, d), rnd(91, Nk, d), rnd(92, Nk, d)
     Oc, lc = forward_head(Q, K, V, 0.4, True)
     On, ln = forward_head(Q, K, V, 0.4, False)
-    np.testing.assert_allclose(Oc, On, atol=1e-14)
-    np.testing.assert_allclose(lc, ln, atol=1e-14)
+    np.testing.assert_allclose(Oc, On, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lc, ln, rtol=0, atol=1e-14)
 
 
 def test_bottom_right_causal_row_equals_noncausal_over_its_visible_keys():
@@ -297,7 +297,7 @@ def test_bottom_right_causal_row_equals_noncausal_over_its_visible_keys():
     for i in range(Nq):
         vis = i + Nk - Nq + 1
         Op, lp = forward_head(Q[i:i + 1], K[:vis], V[:vis], 0.7, False)
-        np.testing.assert_allclose(O[i], Op[0], atol=1e-14)
+        np.testing.assert_allclose(O[i], Op[0], rtol=0, atol=1e-14)
         assert abs(l[i] - lp[0]) < 1e-13
 
 
@@ -320,8 +320,8 @@ def test_key_split_merge_rule(causal):
     Ls = np.stack([p[1] for p in parts])
     Lm = np.log(np.exp(Ls - Ls.max(0)).sum(0)) + Ls.max(0)
     Om = sum(np.exp(p[1] - Lm)[:, None] * p[0] for p in parts)
-    np.testing.assert_allclose(Om, O, atol=1e-13)
-    np.testing.assert_allclose(Lm, L, atol=1e-13)
+    np.testing.assert_allclose(Om, O, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(Lm, L, rtol=0, atol=1e-13)
 
 
 # ---------------------------------------------------------------- block-sparse reference
@@ -333,8 +333,8 @@ def test_block_sparse_all_ones_is_dense():
     for causal in (False, True):
         O, L = oracle.forward_head_block_sparse(Q, K, V, 0.3, causal, m)
         Od, Ld = forward_head(Q, K, V, 0.3, causal)
-        np.testing.assert_allclose(O, Od, atol=1e-13)
-        np.testing.assert_allclose(L, Ld, atol=1e-13)
+        np.testing.assert_allclose(O, Od, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(L, Ld, rtol=0, atol=1e-13)
 
 
 def test_block_diagonal_mask_is_independent_blocks():
@@ -345,8 +345,8 @@ def test_block_diagonal_mask_is_independent_blocks():
     for a in range(0, N, 128):
         b = min(N, a + 128)
         Ob, Lb = forward_head(Q[a:b], K[a:b], V[a:b], 0.3, False)
-        np.testing.assert_allclose(O[a:b], Ob, atol=1e-13)
-        np.testing.assert_allclose(L[a:b], Lb, atol=1e-13)
+        np.testing.assert_allclose(O[a:b], Ob, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(L[a:b], Lb, rtol=0, atol=1e-13)
 
 
 def test_block_sparse_empty_rows_and_brute_force():
@@ -359,7 +359,7 @@ def test_block_sparse_empty_rows_and_brute_force():
         keys = [j for j in range(N) if m[i // 128, j // 128]]
         s = np.array([0.5 * Q[i] @ K[j] for j in keys])
         p = np.exp(s - s.max()) / np.exp(s - s.max()).sum()
-        np.testing.assert_allclose(O[i], p @ V[keys], atol=1e-13)
+        np.testing.assert_allclose(O[i], p @ V[keys], rtol=0, atol=1e-13)
         assert abs(L[i] - (s.max() + np.log(np.exp(s - s.max()).sum()))) < 1e-12
     # causal: block (0,1) lies above the diagonal, so rows 0..127 see nothing
     Oc, Lc = oracle.forward_head_block_sparse(Q, K, V, 0.5, True, m)
