@@ -328,13 +328,7 @@ def run_ours(args, rank, world, local_rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": f"{w.name}: B={B} N={N} H={H} d={d} causal bf16, "
-                                   "q/k/v/dO ~ N(0,1) seed 1003",
-                       "B": B, "N": N, "H": H, "d": d, "causal": True,
-                       "tokens_per_gpu": B * N,
-                       "parallelism": f"replicas x{world} (independent problems per GPU)",
-                       "l2": "no flush: inputs (q,k,v,o,dO = %d MiB) exceed the 126 MB L2"
-                             % (5 * q.numel() * 2 // 2 ** 20)},
+            "config": config_of(w, world),
             "breakdown": {
                 "fwd_ms": round(per_kernel["fwd"], 4), "bwd_pre_ms": round(per_kernel["bwd_pre"], 4),
                 "bwd_main_ms": round(per_kernel["bwd_main"], 4),
@@ -366,6 +360,17 @@ def workload(N: int):
     if N == 65536:
         return synthetic.long_context()
     return synthetic.fwdbwd(N)
+
+
+def config_of(w, world: int) -> dict:
+    """The JSON line's `config` for workload `w` on `world` ranks; both arms print it."""
+    nbytes = 5 * w.B * w.N * w.H * w.d * 2  # q, k, v, o, dO in bf16
+    return {"workload": f"{w.name}: B={w.B} N={w.N} H={w.H} d={w.d} causal bf16, "
+                        f"q/k/v/dO ~ N(0,1) seed {w.seed}",
+            "B": w.B, "N": w.N, "H": w.H, "d": w.d, "causal": True,
+            "tokens_per_gpu": w.B * w.N,
+            "parallelism": f"replicas x{world} (independent problems per GPU)",
+            "l2": "no flush: inputs (q,k,v,o,dO = %d MiB) exceed the 126 MB L2" % (nbytes // 2 ** 20)}
 
 
 # ------------------------------------------------------------------ the oracle on the host
@@ -425,8 +430,7 @@ def run_reference(args, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * secs / args.steps, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{w.name}: B={w.B} N={w.N} H={w.H} d={w.d} causal bf16 inputs",
-                       "B": w.B, "N": w.N, "H": w.H, "d": w.d, "causal": True},
+            "config": config_of(w, world),
             "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0,

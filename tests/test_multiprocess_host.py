@@ -68,6 +68,11 @@ def test_reference_arm_prints_one_json_line_on_rank0_only(tmp_path):
     assert d["impl"] == "reference" and d["unit"] == "TFLOPS" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+    # Same metric, unit, direction and workload description as the CUDA arm's line.
+    import bench
+    assert d["metric"] == bench.METRIC
+    assert d["config"] == bench.config_of(bench.workload(4096), 1)
+    assert d["higher_is_better"] is True and d["unit"] == bench.UNIT
     # a non-zero rank prints nothing and exits cleanly
     env.update(RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
