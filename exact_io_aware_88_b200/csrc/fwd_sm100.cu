@@ -746,8 +746,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 q_released = true;
               }
             };
-            if (cur0 < 0) umma_commit(&bars->o_done[0]);  // nothing accumulated: done
-            if (cur1 < 0) umma_commit(&bars->o_done[1]);
+            // A tile with no active key tile has nothing to accumulate: its O is signalled done
+            // at once, but only after its softmax warpgroup has read the previous unit's O.
+            // Without that wait o_done could complete twice (the previous unit's last PV and
+            // this commit track the same products) before the warpgroup polls it, and a wait
+            // on a phase's parity cannot tell two completions from none.
+            if (cur0 < 0) {
+              if (units > 0 &&
+                  !(ok = mbar_wait(&bars->o_free[0], (units - 1) & 1, ab, status, timeout_ns)))
+                break;
+              umma_commit(&bars->o_done[0]);
+            }
+            if (cur1 < 0) {
+              if (units > 0 &&
+                  !(ok = mbar_wait(&bars->o_free[1], (units - 1) & 1, ab, status, timeout_ns)))
+                break;
+              umma_commit(&bars->o_done[1]);
+            }
             int j = cur0 < 0 ? cur1 : (cur1 < 0 ? cur0 : min(cur0, cur1));
             int gu = g;  // ring position of key tile j
             if (j >= 0) {

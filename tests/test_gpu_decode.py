@@ -122,6 +122,21 @@ def test_block_sparse_all_ones_equals_dense_and_empty_rows(fa):
     _bs_case(fa, 1, N, 2, d, False, m, 6101)
 
 
+@pytest.mark.parametrize("d,causal", [(64, False), (128, True)])
+def test_block_sparse_empty_query_tiles_with_several_units_per_cta(fa, d, causal):
+    """More units than SMs (32 heads x 8 query-tile pairs = 256 on 148 persistent CTAs, so
+    most CTAs take two units) with every third query tile seeing no key: a query tile with
+    nothing to accumulate follows, in the same CTA, one that had work, and its empty O must
+    be signalled only after the previous O was read."""
+    N, H = 2048, 32
+    nt = N // 128
+    rng = np.random.default_rng(300 + d)
+    m = (rng.random((nt, nt)) < 0.4).astype(np.uint8)
+    m[np.arange(nt), np.arange(nt)] = 1
+    m[np.arange(nt) % 3 == 1, :] = 0
+    _bs_case(fa, 1, N, H, d, causal, m, 6300 + d)
+
+
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 def test_block_sparse_interleaved_and_odd_tile_counts(fa, d, causal):
