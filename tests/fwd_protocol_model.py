@@ -10,7 +10,9 @@ scheduler picks a random ready actor at each step (the slowest-poller worst case
 run fails on a deadlock, on a wait that returns before its phase completed, or on a data
 hazard: a product reading a K/V/Q tile that is not loaded, a load overwriting a tile that a
 pending product still reads, P read before it was published, S read before it was
-computed, O overwritten before its epilogue read it, or O read before its products ended.
+computed, an S product issued over a P (same TMEM columns) that no PV has read yet, a
+softmax step (which may rescale O) while the previous PV of its tile still runs, O
+overwritten before its epilogue read it, or O read before its products ended.
 
 The roles follow the kernel's issue logic step by step (names as in the kernel), so a
 change to the kernel's barrier protocol must be mirrored here.  Test infrastructure only.
@@ -43,6 +45,8 @@ class Sim:
         self.p_pub = [0, 0]    # P published per tile
         self.pv_done = [0, 0]  # PV executed per tile
         self.pv_issued = [0, 0]
+        self.p_half_pub = [0, 0]
+        self.s_issued = [0, 0]
         self.o_read_units = [0, 0]   # epilogues done per tile
         self.o_unit_pv = [{}, {}]    # unit -> PVs executed
 
@@ -61,11 +65,13 @@ class Sim:
 
 
 def run(mode, masks0, masks1, nkv_list, seed, stages=4, empty_tile_waits_o_free=True,
-        max_steps=200000):
+        split_p=False, max_steps=200000):
     """mode 'dense' (nkv_list: (nkv0, nkv1) per unit) or 'sparse' (masks0 / masks1: the two
     query tiles' sorted active key tiles per unit).  `stages` is the K/V ring depth (2 at
     head dim 128, 4 at 64).  `empty_tile_waits_o_free=False` restores the earlier block-
     sparse issue logic, which signalled an empty tile's O without waiting for o_free.
+    `split_p` (dense only): P is published in two halves (p_half, then p_full) and each half
+    of PV is issued after its half, as on the 8-bit path.
     Returns "ok" or raises Deadlock / Hazard."""
     S_STAGES = stages
     rng = random.Random(seed)
@@ -104,6 +110,11 @@ def run(mode, masks0, masks1, nkv_list, seed, stages=4, empty_tile_waits_o_free=
                 g += 1
 
     def issue_s(t, pos, u):
+        # S_t shares its TMEM columns with P_t: every earlier P_t must already be read by an
+        # issued PV (the pipe runs in issue order).
+        if sim.pv_issued[t] < sim.s_issued[t]:
+            raise Hazard(f"S{t} issued over a P{t} that no PV has read yet")
+        sim.s_issued[t] += 1
         if not sim.k_loaded.get(pos):
             raise Hazard(f"S{t} issued on K pos {pos} not loaded")
         if sim.q_unit != u:
@@ -150,6 +161,10 @@ def run(mode, masks0, masks1, nkv_list, seed, stages=4, empty_tile_waits_o_free=
                 if j < n0:
                     if j == 0 and u > 0:
                         yield ("wait", "o_free0", u - 1)
+                    if split_p:
+                        yield ("wait", "p_half0", np_[0])
+                        if sim.p_half_pub[0] <= sim.pv_issued[0]:
+                            raise Hazard("first half of PV0 issued before its half of P")
                     yield ("wait", "p_full0", np_[0])
                     issue_pv(0, g + j, u, j == 0)
                     np_[0] += 1
@@ -159,6 +174,10 @@ def run(mode, masks0, masks1, nkv_list, seed, stages=4, empty_tile_waits_o_free=
                         commit("o_done0")
                 if j == 0 and u > 0:
                     yield ("wait", "o_free1", u - 1)
+                if split_p:
+                    yield ("wait", "p_half1", np_[1])
+                    if sim.p_half_pub[1] <= sim.pv_issued[1]:
+                        raise Hazard("first half of PV1 issued before its half of P")
                 yield ("wait", "p_full1", np_[1])
                 issue_pv(1, g + j, u, j == 0)
                 np_[1] += 1
@@ -271,7 +290,14 @@ def run(mode, masks0, masks1, nkv_list, seed, stages=4, empty_tile_waits_o_free=
                 ns += 1
                 if sim.s_done[t] < ns:
                     raise Hazard(f"softmax{t} read S before it was computed")
-                # P overwrites S in place; publish
+                # A step may rescale O in place: the previous step's PV must have landed.
+                if sim.pv_done[t] < ns - 1:
+                    raise Hazard(f"softmax{t} may rescale O while PV{t} of its last step runs")
+                # P overwrites S in place; publish (in two halves on the split path)
+                if split_p:
+                    sim.p_half_pub[t] += 1
+                    sim.complete(f"p_half{t}")
+                    yield ("step",)
                 sim.p_pub[t] += 1
                 sim.complete(f"p_full{t}")
             yield ("wait", f"o_done{t}", u)
@@ -338,7 +364,7 @@ def run(mode, masks0, masks1, nkv_list, seed, stages=4, empty_tile_waits_o_free=
                          f"completed {sim.completed(w[1])})")
         try:
             req = next(roles[c])
-            pending[c] = req
+            pending[c] = None if req[0] == "step" else req
         except StopIteration:
             finished.add(c)
             pending[c] = None

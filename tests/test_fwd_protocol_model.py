@@ -25,9 +25,11 @@ def _random_masks(rng, units, nt, causal, density):
     return m0, m1
 
 
-@pytest.mark.parametrize("stages", [2, 4])
-def test_dense_issue_order_is_safe(stages):
-    rng = random.Random(stages)
+@pytest.mark.parametrize("stages,split_p", [(2, False), (4, False), (4, True)])
+def test_dense_issue_order_is_safe(stages, split_p):
+    """Dense order (head dim 128: 2 stages; 64: 4 stages; 8-bit: 4 stages with P published
+    in halves)."""
+    rng = random.Random(stages + 10 * split_p)
     for case in range(200):
         nkv = []
         for _ in range(rng.randrange(1, 5)):
@@ -35,7 +37,7 @@ def test_dense_issue_order_is_safe(stages):
             nkv.append((a, a + rng.randrange(0, 2)))  # causal pairs: tile 1 sees one more
         for sched in range(4):
             assert model.run("dense", None, None, nkv, seed=100 * case + sched,
-                             stages=stages) == "ok"
+                             stages=stages, split_p=split_p) == "ok"
 
 
 @pytest.mark.parametrize("stages", [2, 4])
