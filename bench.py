@@ -386,6 +386,18 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo; "unknown" elsewhere)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def oracle_sample(t, w, b: int, h: int, n_rows: int):
     """fwd + bwd of one head of the workload, truncated to its first n_rows positions.
     Under the causal mask that prefix is itself an exact attention problem.  Returns
@@ -404,7 +416,7 @@ def cpu_baseline(w, t):
     n_rows = min(w.N, 16384)
     dt, flops = oracle_sample(t, w, 0, 0, n_rows)
     return {"value": round(flops / dt / 1e12, 5), "unit": UNIT, "cores": blas_threads(),
-            "kind": "oracle",
+            "cpu_count": os.cpu_count(), "cpu_model": cpu_model(), "kind": "oracle",
             "sample": f"head (b=0,h=0) of the workload, first {n_rows} positions, fwd+bwd "
                       f"(fp64 numpy, S and P materialised); {dt:.1f} s"}
 
@@ -432,6 +444,7 @@ def run_reference(args, rank, world):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(w, world),
             "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores,
+                             "cpu_count": os.cpu_count(), "cpu_model": cpu_model(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}

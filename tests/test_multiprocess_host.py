@@ -67,6 +67,7 @@ def test_reference_arm_prints_one_json_line_on_rank0_only(tmp_path):
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "TFLOPS" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["cpu_count"] >= 1 and isinstance(d["cpu_baseline"]["cpu_model"], str)
     assert d["e2e"]["h2d_bytes_per_step"] == 0
     # Same metric, unit, direction and workload description as the CUDA arm's line.
     import bench
