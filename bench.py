@@ -418,7 +418,9 @@ def cpu_baseline(w, t):
     return {"value": round(flops / dt / 1e12, 5), "unit": UNIT, "cores": blas_threads(),
             "cpu_count": os.cpu_count(), "cpu_model": cpu_model(), "kind": "oracle",
             "sample": f"head (b=0,h=0) of the workload, first {n_rows} positions, fwd+bwd "
-                      f"(fp64 numpy, S and P materialised); {dt:.1f} s"}
+                      f"(fp64 numpy, S and P materialised); {dt:.1f} s",
+            # Every head costs the same, and a causal prefix of n rows costs ~n^2.
+            "full_workload_s_extrapolated": round(dt * w.B * w.H * (w.N / n_rows) ** 2, 1)}
 
 
 def run_reference(args, rank, world):
