@@ -37,8 +37,8 @@ METRIC = "attention fwd/bwd TFLOPS on 1 B200 vs BF16 tensor-core peak (fraction 
 UNIT = "TFLOPS"
 L2_BYTES = 126 * 2 ** 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# NVIDIA's dense (no 2:4 sparsity) BF16 tensor-core figure for one B200, as given in the
-# hardware notes this build was made with (the datasheet itself is not reachable offline).
+# NVIDIA's published dense (no 2:4 sparsity) BF16 tensor-core figure for one B200, half of
+# the sparse figure it quotes per 8-GPU system (the datasheet is not reachable offline).
 NOMINAL_DENSE_BF16_TFLOPS = 2250.0
 KERNELS_PER_STEP = 4  # fwd, bwd_pre, bwd_main, dq_convert
 
