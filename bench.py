@@ -41,6 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the sparse figure it quotes per 8-GPU system (the datasheet is not reachable offline).
 NOMINAL_DENSE_BF16_TFLOPS = 2250.0
 KERNELS_PER_STEP = 4  # fwd, bwd_pre, bwd_main, dq_convert
+# A timed region at least this long is compared with the sustained (power-capped) peak.
+SUSTAINED_REGION_MS = 1000.0
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -223,7 +225,8 @@ def run_ours(args, rank, world, local_rank):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
-    check(fa.fa_read_device_status(stream), "device status")
+    check(fa.fa_read_device_status(None, stream), "device status")
+    check(fa.fa_read_device_status(ws, stream), "backward status")
 
     # ---- device-resident timed region: K steps, events around each kernel.
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
@@ -240,9 +243,12 @@ def run_ours(args, rank, world, local_rank):
     barrier(world)
     total_ms = max_over_ranks(start.elapsed_time(end), world, dev)
     clocks = clk.summary()
-    check(fa.fa_read_device_status(stream), "device status")
-    per_kernel = {nm: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
-                  for i, nm in enumerate(["fwd", "bwd_pre", "bwd_main", "dq_convert"])}
+    check(fa.fa_read_device_status(None, stream), "device status")
+    check(fa.fa_read_device_status(ws, stream), "backward status")
+    names = ["fwd", "bwd_pre", "bwd_main", "dq_convert"]
+    per_step = {nm: [e[i].elapsed_time(e[i + 1]) for e in evs] for i, nm in enumerate(names)}
+    per_kernel = {nm: statistics.mean(v) for nm, v in per_step.items()}
+    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
 
     # ---- end to end through the public API with host buffers (pinned), copies included.
     # Every step copies its inputs host -> device, runs fa_fwd and fa_bwd, and copies all
@@ -304,7 +310,8 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
     h2d = sum(x.numel() * x.element_size() for x in hin[0].values())
     d2h = sum(x.numel() * x.element_size() for x in hout[0].values())
-    check(fa.fa_read_device_status(stream), "device status")
+    check(fa.fa_read_device_status(None, stream), "device status")
+    check(fa.fa_read_device_status(ws, stream), "backward status")
     del din[1], dout[1]
 
     ms_step = total_ms / args.steps
@@ -313,6 +320,14 @@ def run_ours(args, rank, world, local_rank):
     peaks, peak_src = measured_peaks()
     peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    # The burst peak (a best-of-10 matmul) is the denominator for a timed region shorter than
+    # a second; the sustained one (matmuls back to back for seconds, under the power cap) for
+    # a longer one, whose clocks have settled.
+    long_region = total_ms >= SUSTAINED_REGION_MS
+    peak = peak_sus if long_region else peak_burst
+    peak_kind = (f"{peak_src} bf16 {'sustained' if long_region else 'burst'} "
+                 f"(timed region {total_ms:.0f} ms {'>=' if long_region else '<'} "
+                 f"{SUSTAINED_REGION_MS:.0f} ms)")
     main_tflops = w.bwd_flops() / (per_kernel["bwd_main"] * 1e-3) / 1e12
     fwd_tflops = w.fwd_flops() / (per_kernel["fwd"] * 1e-3) / 1e12
     wl = f"fwdbwd_d128_N{N}"
@@ -329,22 +344,15 @@ def run_ours(args, rank, world, local_rank):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": config_of(w, world),
-            "breakdown": {
-                "fwd_ms": round(per_kernel["fwd"], 4), "bwd_pre_ms": round(per_kernel["bwd_pre"], 4),
-                "bwd_main_ms": round(per_kernel["bwd_main"], 4),
-                "dq_convert_ms": round(per_kernel["dq_convert"], 4),
-                "fwd_tflops": round(fwd_tflops, 1), "bwd_main_tflops": round(main_tflops, 1),
-                "fwd_frac_of_burst_peak": round(fwd_tflops / peak_burst, 4),
-                "bwd_frac_of_burst_peak": round(w.bwd_flops() / ((per_kernel["bwd_pre"] + per_kernel["bwd_main"] + per_kernel["dq_convert"]) * 1e-3) / 1e12 / peak_burst, 4),
-            },
+            "breakdown": breakdown(per_step, step_ms, w, peak_burst),
             "roofline": {"kernel": "bwd_main (fa_bwd_kv)", "bound": "tensor",
-                         "achieved": round(main_tflops, 1), "peak": peak_sus, "unit": "TFLOP/s",
-                         "frac": round(main_tflops / peak_sus, 4),
-                         "peak_kind": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                         "achieved": round(main_tflops, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(main_tflops / peak, 4), "peak_kind": peak_kind,
                          "frac_of_burst_peak": round(main_tflops / peak_burst, 4),
+                         "frac_of_sustained_peak": round(main_tflops / peak_sus, 4),
                          "frac_of_nominal_dense_bf16": round(main_tflops / NOMINAL_DENSE_BF16_TFLOPS, 4),
                          "traffic": traffic},
-            "clocks": clocks,
+            "clocks": clock_record(clocks, ms_step),
             "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 3)},
@@ -354,6 +362,48 @@ def run_ours(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def _stats(v):
+    return {"mean": statistics.mean(v), "median": statistics.median(v), "best": min(v)}
+
+
+def breakdown(per_step, step_ms, w, peak_burst):
+    """Per-kernel device times of the timed steps (mean, median, best of the K steps) and
+    the forward / backward TFLOPS they imply, as fractions of the burst and nominal peaks."""
+    out = {}
+    for nm, v in per_step.items():
+        st = _stats(v)
+        out[f"{nm}_ms"] = round(st["mean"], 4)
+        out[f"{nm}_ms_median"] = round(st["median"], 4)
+        out[f"{nm}_ms_best"] = round(st["best"], 4)
+    st = _stats(step_ms)
+    out["step_ms_median"] = round(st["median"], 4)
+    out["step_ms_best"] = round(st["best"], 4)
+    fwd_med = w.fwd_flops() / (statistics.median(per_step["fwd"]) * 1e-3) / 1e12
+    bwd_steps = [a + b + c for a, b, c in zip(per_step["bwd_pre"], per_step["bwd_main"],
+                                               per_step["dq_convert"])]
+    bwd_med = w.bwd_flops() / (statistics.median(bwd_steps) * 1e-3) / 1e12
+    main_med = w.bwd_flops() / (statistics.median(per_step["bwd_main"]) * 1e-3) / 1e12
+    out["fwd_tflops"] = round(w.fwd_flops() / (statistics.mean(per_step["fwd"]) * 1e-3) / 1e12, 1)
+    out["bwd_main_tflops"] = round(w.bwd_flops() / (statistics.mean(per_step["bwd_main"]) * 1e-3) / 1e12, 1)
+    out["fwd_tflops_median"] = round(fwd_med, 1)
+    out["bwd_tflops_median"] = round(bwd_med, 1)
+    out["bwd_main_tflops_median"] = round(main_med, 1)
+    out["fwd_frac_of_burst_peak"] = round(fwd_med / peak_burst, 4)
+    out["bwd_frac_of_burst_peak"] = round(bwd_med / peak_burst, 4)
+    out["fwd_frac_of_nominal_dense_bf16"] = round(fwd_med / NOMINAL_DENSE_BF16_TFLOPS, 4)
+    out["bwd_frac_of_nominal_dense_bf16"] = round(bwd_med / NOMINAL_DENSE_BF16_TFLOPS, 4)
+    return out
+
+
+def clock_record(clocks, ms_step):
+    """The sampled clock summary plus step time x median SM clock (MHz * ms = kilocycles),
+    which stays comparable across runs whose clocks differ."""
+    c = dict(clocks)
+    if c.get("sm_mhz"):
+        c["step_kcycles_at_median_clock"] = round(ms_step * c["sm_mhz"], 1)
+    return c
 
 
 def workload(N: int):
@@ -529,6 +579,8 @@ def run_sweep(path: str, reps: int = 20, warmup: int = 3):
                                                       w.causal, w.scale, ws, nb, stream)
                 assert det() == 0
                 med, best = timed(det)
+                if fa.fa_read_device_status(ws, stream) != 0:
+                    raise RuntimeError("backward status word reports a failure")
                 rec = {"workload": w.label(), "pass": "bwd_deterministic", "ms": round(med, 4),
                        "ms_best": round(best, 4),
                        "tflops": round(w.bwd_flops() / (med * 1e-3) / 1e12, 1),
@@ -644,7 +696,7 @@ def run_sweep(path: str, reps: int = 20, warmup: int = 3):
             print(json.dumps(rec), file=sys.stderr)
             del q, k, v, q8, k8, vt8, sc, ws, o, lse, t
             torch.cuda.empty_cache()
-    if fa.fa_read_device_status(stream) != 0:
+    if fa.fa_read_device_status(None, stream) != 0:
         raise RuntimeError("device status word reports a timeout")
 
 

@@ -125,6 +125,10 @@ int from_cuda(cudaError_t e) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// A backward workspace starts with the call's status word, in a slot that keeps the parts
+// after it 256-byte aligned.
+constexpr size_t kBwdStatusSlot = 256;
+
 // Split-KV plan: enough (query tile, key slice) units to give every SM of a B200 two (296),
 // at most 64 slices, never more slices than key tiles.  Device-independent, so the
 // workspace size depends on the problem only.
@@ -271,7 +275,8 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (check_shape(B, H, N, d, 1.0f) != FA_OK || d < 1) return 0;
   const size_t rows = static_cast<size_t>(B) * H * N;
   const size_t padded = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128 * 128);
-  return round_up(rows * d * sizeof(float), 256) + 2 * round_up(padded * sizeof(float), 256);
+  return kBwdStatusSlot + round_up(rows * d * sizeof(float), 256) +
+         2 * round_up(padded * sizeof(float), 256);
 }
 
 }  // extern "C"
@@ -281,11 +286,12 @@ namespace {
 enum BwdStage { kStagePre = 1, kStageMain = 2, kStageConvert = 4 };
 
 // Validates the arguments the requested stages use and fills `a`.  Pointers a stage does
-// not use may be null.
+// not use may be null.  With `own_status` the kernels record failures in the workspace's
+// status word (cleared by the preprocess kernel), else in the library-owned word.
 int bwd_prepare(int stages, const void* q, const void* k, const void* v, const void* o,
                 const float* lse, const void* dO, void* dq, void* dk, void* dv, int B, int H,
                 int N, int d, int causal, float scale, void* workspace, size_t workspace_bytes,
-                fa::BwdArgs* a) {
+                fa::BwdArgs* a, bool own_status = true) {
   const bool pre = stages & kStagePre, mid = stages & kStageMain, cvt = stages & kStageConvert;
   if ((pre && (!o || !lse || !dO)) || (mid && (!q || !k || !v || !dO || !dk || !dv)) ||
       (cvt && !dq))
@@ -310,7 +316,8 @@ int bwd_prepare(int stages, const void* q, const void* k, const void* v, const v
     return rc;
   const size_t rows = static_cast<size_t>(B) * H * N;
   const size_t padded = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128 * 128);
-  char* ws = static_cast<char*>(workspace);
+  char* const ws0 = static_cast<char*>(workspace);
+  char* ws = ws0 + kBwdStatusSlot;
   a->o = o;
   a->dO = dO;
   a->lse = lse;
@@ -327,7 +334,8 @@ int bwd_prepare(int stages, const void* q, const void* k, const void* v, const v
   a->d = d;
   a->causal = causal ? 1 : 0;
   a->scale = scale;
-  a->status = di.status;
+  a->status = own_status ? reinterpret_cast<int*>(ws0) : di.status;
+  a->clear_status = own_status;
   a->num_sms = di.num_sms;
   return FA_OK;
 }
@@ -434,7 +442,8 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   if ((rc = noalloc_workspace(&ws))) return rc;
   fa::BwdArgs a;
   rc = bwd_prepare(kStagePre | kStageMain | kStageConvert, q, k, v, o, lse, dO, dq, dk, dv, B, H,
-                   N, d, causal, scale, ws, FA_NOALLOC_WORKSPACE_BYTES, &a);
+                   N, d, causal, scale, ws, FA_NOALLOC_WORKSPACE_BYTES, &a,
+                   /*own_status=*/false);
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = from_cuda(fa::launch_bwd_pre(a, st)))) return rc;
@@ -549,17 +558,19 @@ int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* 
                                       static_cast<cudaStream_t>(stream)));
 }
 
-int fa_read_device_status(int* status_out, void* stream) {
+int fa_read_device_status(const void* status_word_or_null, void* stream) {
+  if (status_word_or_null && !aligned(status_word_or_null, 4)) return FA_ERR_MISALIGNED;
   DeviceInfo di;
   int rc = device_info(&di);
   if (rc) return rc;
+  int* word_ptr = status_word_or_null ? static_cast<int*>(const_cast<void*>(status_word_or_null))
+                                      : di.status;
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
   int word = 0;
   const int zero = 0;
-  if (cudaMemcpy(&word, di.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
-      cudaMemcpy(di.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+  if (cudaMemcpy(&word, word_ptr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(word_ptr, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return FA_ERR_CUDA;
-  if (status_out) *status_out = word;
   return word;
 }
 
@@ -626,12 +637,14 @@ int fa_debug_fwd_schedule(int B, int H, int N, int causal, int grid, int* units,
                                              static_cast<cudaStream_t>(stream)));
 }
 
-int fa_debug_wait_timeout(long long timeout_ns, void* stream) {
+int fa_debug_wait_timeout(long long timeout_ns, void* status_word_or_null, void* stream) {
   if (timeout_ns < 1000 || timeout_ns > 10000000000LL) return FA_ERR_INVALID_ARG;
+  if (status_word_or_null && !aligned(status_word_or_null, 4)) return FA_ERR_MISALIGNED;
   DeviceInfo di;
   int rc = device_info(&di);
   if (rc) return rc;
-  return from_cuda(fa::launch_debug_wait_timeout(static_cast<uint64_t>(timeout_ns), di.status,
+  int* word = status_word_or_null ? static_cast<int*>(status_word_or_null) : di.status;
+  return from_cuda(fa::launch_debug_wait_timeout(static_cast<uint64_t>(timeout_ns), word,
                                                  static_cast<cudaStream_t>(stream)));
 }
 

@@ -533,9 +533,12 @@ __global__ void __launch_bounds__(256)
     bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
                    const float* __restrict__ lse, float* __restrict__ delta,
                    float* __restrict__ lse2, float* __restrict__ dq_acc, int B, int H, int N,
-                   int n_pad, long long acc_vec4, int row_blocks) {
+                   int n_pad, long long acc_vec4, int row_blocks, int* clear_status) {
   constexpr int kTPR = D / 8;           // threads per row
   constexpr int kRowsPerBlock = 256 / kTPR;
+  // The call's own status word (in its workspace) starts out clear; the kernels after this
+  // one in the stream record their failures into it.
+  if (clear_status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *clear_status = FA_OK;
   if (static_cast<int>(blockIdx.x) < row_blocks) {
     const long long rows = static_cast<long long>(B) * N * H;  // rows in memory order (b, n, h)
     const long long row = static_cast<long long>(blockIdx.x) * kRowsPerBlock + threadIdx.x / kTPR;
@@ -619,7 +622,8 @@ static cudaError_t launch_pre_t(const BwdArgs& a, cudaStream_t st) {
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   bwd_pre_kernel<D><<<static_cast<unsigned>(grid), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse,
-      a.delta, a.lse2, a.dq_acc, a.B, a.H, a.N, n_pad, acc_vec4, static_cast<int>(row_blocks));
+      a.delta, a.lse2, a.dq_acc, a.B, a.H, a.N, n_pad, acc_vec4, static_cast<int>(row_blocks),
+      a.clear_status ? a.status : nullptr);
   return cudaGetLastError();
 }
 

@@ -38,7 +38,8 @@ struct BwdArgs {
   float* lse2;    // [B][H][n_pad] fp32 workspace: lse * log2(e)
   int B, H, N, d, causal;
   float scale;
-  int* status;
+  int* status;               // the call's word (workspace) or the library-owned one
+  bool clear_status = false;  // the preprocess kernel clears *status (a workspace word)
   int num_sms;
 };
 

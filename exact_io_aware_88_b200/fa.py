@@ -84,7 +84,7 @@ _lib.fa_fwd_fp8.argtypes = [_P] * 6 + [_I] * 5 + [_F, _P]
 _lib.fa_fwd_fp8.restype = _I
 _lib.fa_fwd_f32.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.fa_fwd_f32.restype = _I
-_lib.fa_read_device_status.argtypes = [ctypes.POINTER(_I), _P]
+_lib.fa_read_device_status.argtypes = [_P, _P]
 _lib.fa_read_device_status.restype = _I
 _lib.fa_status_string.argtypes = [_I]
 _lib.fa_status_string.restype = ctypes.c_char_p
@@ -94,7 +94,7 @@ _lib.fa_debug_umma_tile.argtypes = [_P, _P, _P, _I, _I, _I, _P]
 _lib.fa_debug_umma_tile.restype = _I
 _lib.fa_debug_exp2.argtypes = [_P, _P, _P, _I, _P]
 _lib.fa_debug_exp2.restype = _I
-_lib.fa_debug_wait_timeout.argtypes = [ctypes.c_longlong, _P]
+_lib.fa_debug_wait_timeout.argtypes = [ctypes.c_longlong, _P, _P]
 _lib.fa_debug_wait_timeout.restype = _I
 _lib.fa_debug_tma_tile.argtypes = [_P, _P] + [_I] * 8 + [_P]
 _lib.fa_debug_tma_tile.restype = _I
@@ -235,9 +235,10 @@ def fa_fwd_f32(q, k, v, o, lse, B, H, N, d, causal, scale, stream=None) -> int:
                            int(causal), float(scale), _stream(stream))
 
 
-def fa_read_device_status(stream=None) -> int:
-    word = _I(0)
-    return _lib.fa_read_device_status(ctypes.byref(word), _stream(stream))
+def fa_read_device_status(status_word=None, stream=None) -> int:
+    """Synchronises `stream` and returns (and clears) a device status word: the library-owned
+    one when `status_word` is None, else the word at the start of a backward workspace."""
+    return _lib.fa_read_device_status(_ptr(status_word), _stream(stream))
 
 
 def fa_debug_umma_tile(a, b, c, n, k, mode, stream=None) -> int:
@@ -261,8 +262,8 @@ def fa_debug_fwd_schedule(B, H, N, causal, grid, units, max_rounds, stream=None)
                                       _stream(stream))
 
 
-def fa_debug_wait_timeout(timeout_ns, stream=None) -> int:
-    return _lib.fa_debug_wait_timeout(int(timeout_ns), _stream(stream))
+def fa_debug_wait_timeout(timeout_ns, status_word=None, stream=None) -> int:
+    return _lib.fa_debug_wait_timeout(int(timeout_ns), _ptr(status_word), _stream(stream))
 
 
 # ------------------------------------------------------------------ tensor conveniences

@@ -29,12 +29,21 @@
  *  - Return value: FA_OK (0) on success, else an fa_status code.  On any non-zero return
  *    nothing was launched and no output was touched.  No C++ exception crosses the ABI.
  *  - Device-side failures (a bounded wait inside a kernel that ran out) do not trap the
- *    GPU: the kernel records FA_ERR_TIMEOUT in a library-owned device status word, tears
- *    its CTA down cleanly and returns; read it with fa_read_device_status().  At the end
- *    of every CTA the main forward kernel (fa_fwd, fa_fwd_block_sparse, fa_fwd_fp8) and the
+ *    GPU: the kernel records FA_ERR_TIMEOUT in a device status word, tears its CTA down
+ *    cleanly and returns; read the word with fa_read_device_status().  At the end of every
+ *    CTA the main forward kernel (fa_fwd, fa_fwd_block_sparse, fa_fwd_fp8) and the
  *    backward's key-tile kernel (fa_bwd, fa_bwd_kv) also check that their warp roles agree
  *    on the work done (tiles loaded = consumed, steps per role) and record FA_ERR_INTERNAL
  *    if not.
+ *  - Which status word.  The backward entry points that take a workspace (fa_bwd,
+ *    fa_bwd_deterministic and the staged fa_bwd_preprocess / fa_bwd_kv / fa_bwd_dq_convert)
+ *    record into a word of their own: the first 4 bytes of that workspace, cleared when the
+ *    call's first kernel starts.  Every other entry point (the forward family, fa_bwd_noalloc,
+ *    the self-tests) records into one library-owned word per device.  Calls on several
+ *    streams at once therefore each get their own backward word (one workspace per
+ *    concurrent call, as the dQ accumulator already requires), while the library word is
+ *    shared: it holds the first failure of any of those calls, whichever stream it came
+ *    from, and reading it clears it for every caller.
  */
 #ifndef FA_H_
 #define FA_H_
@@ -66,10 +75,11 @@ typedef enum {
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            int B, int H, int N, int d, int causal, float scale, void* stream);
 
-/* Bytes of device workspace fa_bwd needs for this problem: an fp32 dQ accumulator
- * (B*H*N*d floats), then the fp32 row statistic D and the base-2 logsumexp, each
- * B*H*Np floats with Np = N rounded up to a multiple of 128; every part starts on a
- * 256-byte boundary.  Returns 0 if the arguments are invalid. */
+/* Bytes of device workspace fa_bwd needs for this problem: the call's status word (an int
+ * at offset 0, in a 256-byte slot), an fp32 dQ accumulator (B*H*N*d floats), then the fp32
+ * row statistic D and the base-2 logsumexp, each B*H*Np floats with Np = N rounded up to a
+ * multiple of 128; every part starts on a 256-byte boundary.  Returns 0 if the arguments
+ * are invalid. */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
 /* Backward pass.  Inputs are the forward's q, k, v, its outputs o and lse, and the
@@ -77,7 +87,8 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
  * aligned here).  Writes dq, dk, dv
  * ([B][N][H][d] bf16).  `workspace` is caller-owned device memory of at least
  * fa_bwd_workspace_bytes(B, H, N, d) bytes, 256-byte aligned; its contents on entry are
- * ignored and on return are unspecified.  d must be 64 or 128.
+ * ignored and on return are unspecified except for its first int, the call's status word
+ * (read it with fa_read_device_status(workspace, stream)).  d must be 64 or 128.
  * Steps: D = rowsum(dO o O) with dQ-accumulator clearing; per key/value tile, recompute
  * S^T and P^T from lse, dP^T = V dO^T, dS^T = P^T o (dP^T - D); dV += P^T dO and
  * dK += dS^T Q accumulate in TMEM; dQ += dS K is reduced in fp32 into the workspace
@@ -101,7 +112,8 @@ int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void
 /* The three stages fa_bwd runs, exposed so a caller can time or schedule them apart.
  * Calling them in this order on one stream with the same workspace is exactly fa_bwd.
  *  fa_bwd_preprocess: D = rowsum(dO o O) and lse*log2(e) into the workspace; clears the
- *                     workspace's fp32 dQ accumulator.  Reads o, lse, dO.
+ *                     workspace's fp32 dQ accumulator and its status word.  Reads o, lse,
+ *                     dO.
  *  fa_bwd_kv:         the recompute kernel: per key/value tile, rebuilds S^T and P^T from
  *                     the workspace statistics, writes dk, dv and adds dS K into the dQ
  *                     accumulator.  Reads q, k, v, dO; needs fa_bwd_preprocess first.
@@ -133,7 +145,12 @@ int fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, void* w
  *  - Every call on a device shares the one array.  Calls whose work overlaps on the GPU
  *    (e.g. on two streams without ordering between them) race on it and give wrong
  *    results; serialise them.  Each call re-initialises what it needs (the dQ accumulator
- *    is cleared), so leftovers of a previous call do not matter. */
+ *    is cleared), so leftovers of a previous call do not matter.
+ *  - The device address found at set-up is cached per device for the life of the process.
+ *    It stays valid as long as that device's primary context does: a caller that destroys
+ *    the context (cudaDeviceReset) must not call this entry point on that device again.
+ *  - A failure inside a kernel is recorded in the library-owned status word (read it with
+ *    fa_read_device_status(NULL, stream)). */
 #define FA_NOALLOC_WORKSPACE_BYTES (64u * 1024u * 1024u)
 int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                    const void* dO, void* dq, void* dk, void* dv,
@@ -215,10 +232,15 @@ int fa_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* sca
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
                int B, int H, int N, int d, int causal, float scale, void* stream);
 
-/* Synchronises `stream`, then returns and clears the library's device status word
- * (FA_OK, FA_ERR_TIMEOUT or FA_ERR_INTERNAL; the first failure recorded wins).  If
- * `status_out` is non-null the raw word is also stored there (host pointer).  Returns FA_ERR_CUDA if the synchronisation itself failed. */
-int fa_read_device_status(int* status_out, void* stream);
+/* Synchronises `stream`, then returns and clears a device status word: FA_OK, or the
+ * first failure recorded there (FA_ERR_TIMEOUT, FA_ERR_INTERNAL, FA_ERR_UNSUPPORTED).
+ *   status_word_or_null : NULL for the library-owned word of the current device, or the
+ *       DEVICE pointer of a backward call's own word, which is the start of the workspace
+ *       that call was given (4-byte aligned, else FA_ERR_MISALIGNED).
+ * `stream` must be the stream (or a stream ordered after the one) the calls of
+ * interest ran on.  Returns FA_ERR_CUDA if the synchronisation or the copy failed (no
+ * kernel ever records that code, so it cannot be confused with a word's value). */
+int fa_read_device_status(const void* status_word_or_null, void* stream);
 
 /* Static, human-readable name of a status code. */
 const char* fa_status_string(int status);

@@ -51,9 +51,11 @@ int fa_debug_fwd_schedule(int B, int H, int N, int causal, int grid, int* units,
 
 /* Launches one CTA whose only work is a bounded wait on an mbarrier that nothing ever
  * arrives at.  The wait gives up after `timeout_ns` nanoseconds (1e3 .. 1e10), records
- * FA_ERR_TIMEOUT in the device status word and the CTA exits normally.  Read the result
- * with fa_read_device_status(). */
-int fa_debug_wait_timeout(long long timeout_ns, void* stream);
+ * FA_ERR_TIMEOUT in a status word and the CTA exits normally.  status_word_or_null: NULL
+ * for the library-owned word, or a backward workspace (its first int is that call's word,
+ * see fa_read_device_status), 4-byte aligned.  Read the result with
+ * fa_read_device_status() on the same word. */
+int fa_debug_wait_timeout(long long timeout_ns, void* status_word_or_null, void* stream);
 
 #ifdef __cplusplus
 }

@@ -39,12 +39,13 @@ int main(void) {
   }
   CHECK(strcmp(fa_status_string(4242), "unknown status") == 0);
 
-  /* Backward workspace: fp32 dQ accumulator + D + log2-scaled LSE, each 256-byte padded. */
+  /* Backward workspace: the call's status word (256-byte slot), fp32 dQ accumulator, D and
+   * the log2-scaled LSE, each 256-byte padded. */
   {
     const int B = 2, H = 3, N = 1000, d = 64;
     const size_t rows = (size_t)B * H * N;
     const size_t padded = (size_t)B * H * ((N + 127) / 128 * 128);
-    CHECK(fa_bwd_workspace_bytes(B, H, N, d) == up256(rows * d * 4) + 2 * up256(padded * 4));
+    CHECK(fa_bwd_workspace_bytes(B, H, N, d) == 256 + up256(rows * d * 4) + 2 * up256(padded * 4));
     CHECK(fa_bwd_workspace_bytes(0, H, N, d) == 0);
     CHECK(fa_bwd_workspace_bytes(B, H, -1, d) == 0);
   }
@@ -94,6 +95,9 @@ int main(void) {
   /* FP8 forward: head dim 128 only. */
   CHECK(fa_fwd_fp8(A16, A16, A16, A16, A16, A16, 1, 1, 256, 64, 0, 0.1f, NULL) ==
         FA_ERR_UNSUPPORTED);
+
+  /* A status word must be 4-byte aligned; checked before the device is touched. */
+  CHECK(fa_read_device_status(AT(2), NULL) == FA_ERR_MISALIGNED);
 
   if (failures == 0) printf("c abi: all checks passed\n");
   return failures == 0 ? 0 : 1;

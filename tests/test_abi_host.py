@@ -9,6 +9,11 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
+@pytest.fixture(autouse=True)
+def _host_only(no_visible_gpu):
+    """Every call below passes fake device addresses (see no_visible_gpu)."""
+
+
 @pytest.fixture(scope="module")
 def fa():
     import __graft_entry__
@@ -48,7 +53,8 @@ def test_workspace_size_formula(fa):
     for B, H, N, d in [(1, 16, 4096, 128), (2, 3, 1000, 64), (1, 1, 1, 64)]:
         rows = B * H * N
         padded = B * H * ((N + 127) // 128 * 128)
-        assert fa.fa_bwd_workspace_bytes(B, H, N, d) == up(rows * d * 4) + 2 * up(padded * 4)
+        # status word slot + dQ accumulator + D + base-2 logsumexp
+        assert fa.fa_bwd_workspace_bytes(B, H, N, d) == 256 + up(rows * d * 4) + 2 * up(padded * 4)
     assert fa.fa_bwd_workspace_bytes(0, 1, 1, 64) == 0
     assert fa.fa_bwd_workspace_bytes(1, 1, -5, 64) == 0
 
@@ -145,3 +151,5 @@ def test_debug_entry_points_reject_bad_arguments(fa):
     assert fa.fa_debug_umma_tile(A16, A16, A16, 96, 64, 0, stream=0) == fa.FA_ERR_UNSUPPORTED
     assert fa.fa_debug_umma_tile(A16, A16, A16, 64, 64, 3, stream=0) == fa.FA_ERR_UNSUPPORTED
     assert fa.fa_debug_wait_timeout(10, stream=0) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_debug_wait_timeout(10_000, A16 + 2, stream=0) == fa.FA_ERR_MISALIGNED
+    assert fa.fa_read_device_status(A16 + 2, stream=0) == fa.FA_ERR_MISALIGNED

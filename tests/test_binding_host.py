@@ -6,6 +6,11 @@ import pytest
 import torch
 
 
+@pytest.fixture(autouse=True)
+def _host_only(no_visible_gpu):
+    """The wrappers must refuse every case below before a CUDA call (see no_visible_gpu)."""
+
+
 @pytest.fixture(scope="module")
 def fa():
     import __graft_entry__

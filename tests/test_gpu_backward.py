@@ -21,12 +21,20 @@ def fa():
     return mod
 
 
+def _workspace(fa, q):
+    B, N, H, d = q.shape
+    return torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), device=q.device, dtype=torch.uint8)
+
+
 def _run(fa, t, causal, scale):
     q, k, v, dO = cuda(t, ("q", "k", "v", "dO"))
     o, lse = fa.attention_forward(q, k, v, causal=causal, scale=scale)
-    dq, dk, dv = fa.attention_backward(q, k, v, o, lse, dO, causal=causal, scale=scale)
+    ws = _workspace(fa, q)
+    dq, dk, dv = fa.attention_backward(q, k, v, o, lse, dO, causal=causal, scale=scale,
+                                       workspace=ws)
     torch.cuda.synchronize()
-    assert fa.fa_read_device_status() == 0
+    assert fa.fa_read_device_status() == 0      # the forward's (library-owned) word
+    assert fa.fa_read_device_status(ws) == 0    # the backward call's own word
     return dq, dk, dv
 
 
@@ -103,9 +111,12 @@ def test_deterministic_backward_parity(fa, B, N, H, d, causal):
     scale = 1.0 / math.sqrt(d)
     q, k, v, dO = cuda(t, ("q", "k", "v", "dO"))
     o, lse = fa.attention_forward(q, k, v, causal=causal, scale=scale)
-    got = fa.attention_backward(q, k, v, o, lse, dO, causal=causal, scale=scale, deterministic=True)
+    ws = _workspace(fa, q)
+    got = fa.attention_backward(q, k, v, o, lse, dO, causal=causal, scale=scale, deterministic=True,
+                                workspace=ws)
     torch.cuda.synchronize()
     assert fa.fa_read_device_status() == 0
+    assert fa.fa_read_device_status(ws) == 0
     refs = oracle.backward(*(synthetic.to_f64(t[n]) for n in ("q", "k", "v", "dO")), scale, causal)
     for name, g, r in zip(("dq", "dk", "dv"), got, refs):
         assert grad_err(to_np(g), r) <= GRAD_REL_L2, (name, grad_err(to_np(g), r))
@@ -130,3 +141,35 @@ def test_deterministic_backward_is_bitwise_repeatable_at_full_size(fa, w):
     Q, K, V, DO = (synthetic.to_f64(t[n][0, :, 0]) for n in ("q", "k", "v", "dO"))
     ref = oracle.dq_rows(Q, K, V, DO, w.scale, w.causal, rows)
     assert rel_l2(to_np(a[0][0, rows, 0]), ref) <= GRAD_REL_L2
+
+
+# ------------------------------------------------------------------ per-call status word
+
+def test_backward_status_word_is_per_call(fa):
+    # Two backward calls run on two streams, each with its own workspace, so each has its
+    # own status word (the workspace's first int).  A bounded wait that runs out on the
+    # first stream, recorded into the first call's word, shows up there only: the second
+    # call's word and the library-owned word stay clear.
+    B, N, H, d = 1, 512, 2, 128
+    scale = 1.0 / math.sqrt(d)
+    t = synthetic.draw(B, N, H, d, 41, "bf16", with_grad=True)
+    q, k, v, dO = cuda(t, ("q", "k", "v", "dO"))
+    o, lse = fa.attention_forward(q, k, v, causal=True, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.fa_read_device_status() == fa.FA_OK
+    streams = (torch.cuda.Stream(), torch.cuda.Stream())
+    wss = (_workspace(fa, q), _workspace(fa, q))
+    outs = [[torch.full_like(q, float("nan")) for _ in range(3)] for _ in range(2)]
+    for s, ws, (dq, dk, dv) in zip(streams, wss, outs):
+        rc = fa.fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, True, scale, ws, ws.numel(),
+                       stream=s)
+        assert rc == fa.FA_OK, fa.status_string(rc)
+    assert fa.fa_debug_wait_timeout(20_000_000, wss[0], stream=streams[0]) == fa.FA_OK
+    assert fa.fa_read_device_status(wss[0], stream=streams[0]) == fa.FA_ERR_TIMEOUT
+    assert fa.fa_read_device_status(wss[1], stream=streams[1]) == fa.FA_OK
+    assert fa.fa_read_device_status() == fa.FA_OK
+    assert fa.fa_read_device_status(wss[0], stream=streams[0]) == fa.FA_OK  # read clears it
+    # Both calls computed the same gradients (dK, dV bit for bit: fixed accumulation order).
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0][1], outs[1][1]) and torch.equal(outs[0][2], outs[1][2])
+    assert rel_l2(to_np(outs[0][0]), to_np(outs[1][0])) <= 1e-3

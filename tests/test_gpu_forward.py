@@ -146,16 +146,30 @@ def test_bf16_forward_gpu_invariants(fa):
     np.testing.assert_array_equal(O[:, 0], V[:, 0])
 
 
-@pytest.mark.parametrize("w", [synthetic.fwd_sweep(64, 4096, False), synthetic.fwd_sweep(128, 16384, True),
-                               synthetic.long_context()], ids=lambda w: w.label())
+# Every (head dim, causal) instantiation of the dense forward runs here at a size where each
+# persistent CTA takes many units (B*H*ceil(N/256) units on at most 148 CTAs), so the hand-over
+# of the O columns and of the K/V ring from one unit to the next is checked against the oracle:
+# d=64 non-causal 4k (1024 units), d=64 causal 16k (2048) and 512 (2048 one-pair units),
+# d=128 non-causal 16k (1024) and 512 (1024), d=128 causal 16k (1024) and 64k (256).
+FULL_SIZE = [synthetic.fwd_sweep(64, 4096, False), synthetic.fwd_sweep(64, 16384, True),
+             synthetic.fwd_sweep(64, 512, True), synthetic.fwd_sweep(128, 16384, False),
+             synthetic.fwd_sweep(128, 512, False), synthetic.fwd_sweep(128, 16384, True),
+             synthetic.long_context()]
+
+
+@pytest.mark.parametrize("w", FULL_SIZE, ids=lambda w: w.label())
 def test_bf16_forward_full_size_sampled_rows(fa, w):
     t = synthetic.draw_workload(w, with_grad=False)
     q, k, v = cuda(t, ("q", "k", "v"))
     o, lse = fa.attention_forward(q, k, v, causal=w.causal, scale=w.scale)
     torch.cuda.synchronize()
+    assert fa.fa_read_device_status() == 0
     rng = np.random.default_rng(w.seed)
-    rows = np.unique(np.concatenate([[0, 1, 127, 128, w.N - 1], rng.integers(0, w.N, 59)]))
-    for b, h in [(0, 0), (w.B - 1, w.H - 1)]:
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, 255, 256, w.N - 1], rng.integers(0, w.N, 57)]))
+    # First and last head, plus two from the middle of the unit order (other batch entries
+    # and heads land on other CTAs and rounds of the persistent schedule).
+    heads = sorted({(0, 0), (w.B - 1, w.H - 1), (w.B // 2, w.H // 3), ((w.B - 1) // 3, w.H - 2)})
+    for b, h in heads:
         Q, K, V = (synthetic.to_f64(t[n][b, :, h]) for n in ("q", "k", "v"))
         O_ref, L_ref = oracle.forward_rows(Q, K, V, w.scale, w.causal, rows)
         O = to_np(o[b, rows, h])

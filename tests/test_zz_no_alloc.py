@@ -23,7 +23,7 @@ def fa():
     return mod
 
 
-def test_oversized_problem_is_refused_before_launch(fa):
+def test_oversized_problem_is_refused_before_launch(fa, no_visible_gpu):
     a16 = 1 << 20  # never dereferenced: the call must fail on the size check
     ptrs = [a16] * 9
     # B*H*N*d*4 bytes of dQ accumulator alone exceed the 64 MiB built-in workspace
