@@ -83,15 +83,17 @@ int check_shape(int B, int H, int N, int d, float scale) {
 // 4-D view [B][N][H][d] (innermost first: d, H, N, B) of a bf16 tensor, tiled in boxes of
 // 64 d-elements (128 bytes, the 128-byte swizzle span) x 1 head x 128 rows x 1 batch.
 // 8-bit tensors (E4M3 codes as UINT8) use boxes of 128 d-elements, again 128 bytes.
+// `box_rows` rows per box (128; the forward's output map uses 32, one warp's rows).
 int encode_bnhd(CUtensorMap* m, const void* ptr, int B, int N, int H, int d,
-                CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+                CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, int box_rows = 128) {
   const cuuint64_t es = (dt == CU_TENSOR_MAP_DATA_TYPE_UINT8) ? 1 : 2;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * es,
                                  static_cast<cuuint64_t>(H) * d * es,
                                  static_cast<cuuint64_t>(N) * H * d * es};
-  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / es), 1, 128, 1};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / es), 1,
+                             static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = g_encode(m, dt, 4, const_cast<void*>(ptr), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -187,9 +189,9 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   if ((rc = device_info(&di))) return rc;
   fa::FwdArgs a;
   if ((rc = encode_bnhd(&a.tm_q, q, B, N, H, d)) || (rc = encode_bnhd(&a.tm_k, k, B, N, H, d)) ||
-      (rc = encode_bnhd(&a.tm_v, v, B, N, H, d)))
+      (rc = encode_bnhd(&a.tm_v, v, B, N, H, d)) ||
+      (rc = encode_bnhd(&a.tm_o, o, B, N, H, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32)))
     return rc;
-  a.o = o;
   a.lse = lse;
   a.B = B;
   a.H = H;
@@ -255,9 +257,9 @@ int fa_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* sca
   const int npad = (N + 15) / 16 * 16;
   if ((rc = encode_bnhd(&a.tm_q, q8, B, N, H, d, CU_TENSOR_MAP_DATA_TYPE_UINT8)) ||
       (rc = encode_bnhd(&a.tm_k, k8, B, N, H, d, CU_TENSOR_MAP_DATA_TYPE_UINT8)) ||
-      (rc = encode_vt8(&a.tm_v, vt8, B, H, d, npad)))
+      (rc = encode_vt8(&a.tm_v, vt8, B, H, d, npad)) ||
+      (rc = encode_bnhd(&a.tm_o, o, B, N, H, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32)))
     return rc;
-  a.o = o;
   a.lse = lse;
   a.scales = scales;
   a.B = B;
@@ -524,9 +526,9 @@ int fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, fl
   if ((rc = device_info(&di))) return rc;
   fa::FwdArgs a;
   if ((rc = encode_bnhd(&a.tm_q, q, B, N, H, d)) || (rc = encode_bnhd(&a.tm_k, k, B, N, H, d)) ||
-      (rc = encode_bnhd(&a.tm_v, v, B, N, H, d)))
+      (rc = encode_bnhd(&a.tm_v, v, B, N, H, d)) ||
+      (rc = encode_bnhd(&a.tm_o, o, B, N, H, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32)))
     return rc;
-  a.o = o;
   a.lse = lse;
   a.block_mask = block_mask;
   a.mask_words = static_cast<uint32_t*>(workspace);

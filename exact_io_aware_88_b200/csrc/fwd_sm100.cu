@@ -88,8 +88,14 @@ struct Cfg {
   // Block-sparse bitmasks: loader (2 tiles), MMA issuer (2), softmax warpgroup 0 and 1.
   static constexpr int kOffMask = kOffBar + kBarBytes;
   static constexpr int kMaskBytes = (2 + 2 + 8) * 32 * 4;  // + one copy per softmax warp
-  static constexpr int kSmemBytes = kOffMask + kMaskBytes;  // base is 1024-aligned (checked)
+  // O epilogue: one staging box per softmax warp (32 rows x 128 bytes, 128-byte swizzled),
+  // written out by TMA stores.
+  static constexpr int kOffStage = kOffMask + kMaskBytes;
+  static constexpr int kStageBytes = 32 * 128;
+  static constexpr int kSmemBytes = kOffStage + 8 * kStageBytes;  // base is 1024-aligned (checked)
   static constexpr uint32_t kColO = 256;  // O_t at kColO + 128 t
+  static_assert(kOffStage % 1024 == 0, "staging boxes need 1024-byte alignment (128-byte swizzle)");
+  static_assert(kSmemBytes <= 232448, "more shared memory than a CTA can have");
 };
 
 struct Bars {
@@ -231,7 +237,7 @@ __device__ __forceinline__ float tree_max(const float* v) {
 template <int D, bool CAUSAL, bool F8, bool SPARSE = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                float* __restrict__ lse, const float* __restrict__ scales,
                const uint32_t* __restrict__ mask_words, int B, int H, int N, float scale_log2,
                int num_pairs, int* status, uint64_t timeout_ns) {
@@ -525,20 +531,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < D; ++i) o[i] = 0u;
       }
-      if (row < N) {
-        const float inv_l = empty ? 0.f : out_mul / l;
-        __nv_bfloat16* orow = out + ((static_cast<size_t>(b) * N + row) * H + h) * D;
-#pragma unroll
-        for (int c8 = 0; c8 < D / 8; ++c8)
-          reinterpret_cast<uint4*>(orow)[c8] = make_uint4(
-              pack_bf16x2(__uint_as_float(o[8 * c8 + 0]) * inv_l, __uint_as_float(o[8 * c8 + 1]) * inv_l),
-              pack_bf16x2(__uint_as_float(o[8 * c8 + 2]) * inv_l, __uint_as_float(o[8 * c8 + 3]) * inv_l),
-              pack_bf16x2(__uint_as_float(o[8 * c8 + 4]) * inv_l, __uint_as_float(o[8 * c8 + 5]) * inv_l),
-              pack_bf16x2(__uint_as_float(o[8 * c8 + 6]) * inv_l, __uint_as_float(o[8 * c8 + 7]) * inv_l));
+      if (row < N)
         lse[static_cast<size_t>(x.bh) * N + row] =
             empty ? -INFINITY : (m + __log2f(l)) * 0.69314718055994531f;
+      // O = O / l in bf16, written as whole 128-byte lines: each warp stages its 32 rows in
+      // boxes of 64 head-dim elements (128-byte swizzle: conflict-free 16-byte shared stores)
+      // and lane 0 hands each box to a TMA store, which clips the rows past N.  Before a box
+      // is refilled, the store that read it must be done reading.
+      const float inv_l = empty ? 0.f : out_mul / l;
+      const int r0 = q0 + (warp & 3) * 32;
+      uint8_t* stage = smem + C::kOffStage + warp * C::kStageBytes;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          const uint32_t* e = &o[64 * c + 8 * p];
+          *reinterpret_cast<uint4*>(stage + sw128_offset(lane, p)) = make_uint4(
+              pack_bf16x2(__uint_as_float(e[0]) * inv_l, __uint_as_float(e[1]) * inv_l),
+              pack_bf16x2(__uint_as_float(e[2]) * inv_l, __uint_as_float(e[3]) * inv_l),
+              pack_bf16x2(__uint_as_float(e[4]) * inv_l, __uint_as_float(e[5]) * inv_l),
+              pack_bf16x2(__uint_as_float(e[6]) * inv_l, __uint_as_float(e[7]) * inv_l));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && r0 < N) {
+          tma_store_4d(&tm_o, stage, 64 * c, h, r0, b);
+          bulk_commit();
+        }
       }
     }
+    // Every O store has completed before the CTA's shared memory goes away.
+    if (lane == 0) bulk_wait_all();
     if ((warp & 3) == 0 && lane == 0) {
       bars->count[4 + t] = ns;
       bars->count[8 + t] = units;
@@ -984,8 +1009,7 @@ static cudaError_t launch_t(const FwdArgs& a, cudaStream_t st) {
   if (units > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const int grid = static_cast<int>(std::min<long long>(units, a.num_sms));
   const float scale_log2 = a.scale * 1.4426950408889634f;
-  kern<<<grid, kThreads, C::kSmemBytes, st>>>(a.tm_q, a.tm_k, a.tm_v,
-                                              static_cast<__nv_bfloat16*>(a.o), a.lse, a.scales,
+  kern<<<grid, kThreads, C::kSmemBytes, st>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_o, a.lse, a.scales,
                                               a.mask_words, a.B, a.H, a.N, scale_log2, num_pairs,
                                               a.status, kDefaultWaitTimeoutNs);
   return cudaGetLastError();

@@ -16,7 +16,7 @@ struct FwdArgs {
   CUtensorMap tm_q, tm_k, tm_v;  // 4-D maps over [B][N][H][d] bf16, box {64,1,128,1}
                                  // (8-bit path: E4M3 box {128,1,128,1}; tm_v over V^T
                                  // [B][H][d][Npad], box {128,128,1,1})
-  void* o;
+  CUtensorMap tm_o;               // 4-D map over the bf16 output [B][N][H][d], box {64,1,32,1}
   float* lse;
   const float* scales = nullptr;  // 8-bit path: [3][B*H] dequantisation scales
   const uint8_t* block_mask = nullptr;  // block-sparse: [ceil(N/128)][ceil(N/128)] bytes

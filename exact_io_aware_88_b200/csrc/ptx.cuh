@@ -111,6 +111,29 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
+// 4-D tiled bulk tensor store this CTA's shared memory -> global, tracked in the issuing
+// thread's bulk-async group.  Coordinates are innermost first and non-negative; the parts of
+// the box past the tensor's extent are not written.  The writes to the source that precede
+// it must be made visible to the async proxy first (fence_proxy_async_smem + a barrier).
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* m, const void* src, int c0, int c1,
+                                             int c2, int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2),
+               "r"(c3)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Until every bulk store this thread committed has finished reading its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Until every bulk store this thread committed has completed (its writes performed).
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // L2 cache-policy operands for the .L2::cache_hint qualifier (createpolicy results).
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t p;
