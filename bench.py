@@ -700,16 +700,40 @@ def run_sweep(path: str, reps: int = 20, warmup: int = 3):
         raise RuntimeError("device status word reports a timeout")
 
 
-KERNEL_CASES = ("fwd_d64_N4096", "fwd_fp8_N4096")
+KERNEL_CASES = ("fwd_d64_N4096", "fwd_fp8_N4096", "fwd_d128_N4096_causal", "bwd_N4096")
 
 
 def run_kernel_case(name: str, launches: int = 4):
-    """A few launches of one kernel on one workload, for a profiler to capture: the head-dim
-    64 forward (fwd_d64, N=4096, non-causal) or the E4M3 forward (N=4096, H=16, d=128,
-    non-causal, after one fa_fp8_quantize).  Prints one line; nothing is timed."""
+    """A few launches of one kernel on one workload, for a profiler to capture (every case
+    holds well under 1 GB on the device, and its inputs exceed the 126 MB L2):
+      fwd_d64_N4096          the head-dim 64 forward (B=4, N=4096, H=32, non-causal);
+      fwd_fp8_N4096          the E4M3 forward (B=4, N=4096, H=16, d=128, non-causal, after
+                             one fa_fp8_quantize);
+      fwd_d128_N4096_causal  the head-dim 128 causal forward (B=4, N=4096, H=16);
+      bwd_N4096              one forward, then `launches` backward passes (fa_bwd: its
+                             three kernels) on the fwd+bwd workload at N=4096 (B=4, H=16,
+                             d=128, causal).
+    Prints one line; nothing is timed."""
     import torch
     from exact_io_aware_88_b200 import fa
-    if name == "fwd_d64_N4096":
+    if name == "fwd_d128_N4096_causal":
+        w = synthetic.fwd_sweep(128, 4096, True)
+        t = synthetic.draw_workload(w)
+        q, k, v = (t[n].cuda() for n in ("q", "k", "v"))
+        for _ in range(launches):
+            fa.attention_forward(q, k, v, causal=True)
+    elif name == "bwd_N4096":
+        w = synthetic.fwdbwd(4096)
+        t = synthetic.draw_workload(w, with_grad=True)
+        q, k, v, dO = (t[n].cuda() for n in ("q", "k", "v", "dO"))
+        o, lse = fa.attention_forward(q, k, v, causal=True)
+        ws = torch.empty(fa.fa_bwd_workspace_bytes(w.B, w.H, w.N, w.d), device="cuda",
+                         dtype=torch.uint8)
+        for _ in range(launches):
+            fa.attention_backward(q, k, v, o, lse, dO, causal=True, workspace=ws)
+        if fa.fa_read_device_status(ws) != 0:
+            raise RuntimeError("backward status word reports a failure")
+    elif name == "fwd_d64_N4096":
         w = synthetic.fwd_sweep(64, 4096, False)
         t = synthetic.draw_workload(w)
         q, k, v = (t[n].cuda() for n in ("q", "k", "v"))
