@@ -314,7 +314,9 @@ int bwd_prepare(int stages, const void* q, const void* k, const void* v, const v
   if (mid && ((rc = encode_bnhd(&a->tm_q, q, B, N, H, d)) ||
               (rc = encode_bnhd(&a->tm_k, k, B, N, H, d)) ||
               (rc = encode_bnhd(&a->tm_v, v, B, N, H, d)) ||
-              (rc = encode_bnhd(&a->tm_do, dO, B, N, H, d))))
+              (rc = encode_bnhd(&a->tm_do, dO, B, N, H, d)) ||
+              (rc = encode_bnhd(&a->tm_dk, dk, B, N, H, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32)) ||
+              (rc = encode_bnhd(&a->tm_dv, dv, B, N, H, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32))))
     return rc;
   const size_t rows = static_cast<size_t>(B) * H * N;
   const size_t padded = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128 * 128);

@@ -119,9 +119,9 @@ template <int D, bool CAUSAL, bool WITH_DQ>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                     const float* __restrict__ lse2, const float* __restrict__ delta,
-                    float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk,
-                    __nv_bfloat16* __restrict__ dv, int B, int H, int N, int n_pad,
+                    float* __restrict__ dq_acc, int B, int H, int N, int n_pad,
                     float scale, float scale_log2, int num_kvtiles, int* status,
                     uint64_t timeout_ns) {
   using C = Cfg<D>;
@@ -278,28 +278,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if ((warp & 3) == 0 && lane == 0) bars->count[3 + half] = steps_done;
     // ---------------------------------------------------------------- dK / dV epilogue
-    // Warpgroup 0 writes dK, warpgroup 1 writes dV.
+    // Warpgroup 0 writes dK (times scale), warpgroup 1 writes dV, as whole 128-byte lines:
+    // each warp stages its 32 key rows in 128-byte-swizzled boxes of 64 head-dim elements in
+    // the Q stages (free once dkdv_done has fired: every product has completed) and lane 0
+    // hands them to TMA stores, which clip the rows past N.
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->dkdv_done, 0, ab, status, timeout_ns));
     if (ok) {
       tc_fence_after();
-      const size_t orow = ((static_cast<size_t>(b) * N + key) * H + h) * D;
       const uint32_t col = half == 0 ? C::kColDK : C::kColDV;
       const float mul = half == 0 ? scale : 1.f;
-      __nv_bfloat16* dst = (half == 0 ? dk : dv) + orow;
+      uint8_t* stage = sQ + warp * (C::kChunks * 4096);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t u[32];
         tmem_ld32(lane_base + col + c * 32, u);
-        if (key < N) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            d4[v4] = make_uint4(
-                pack_bf16x2(__uint_as_float(u[8 * v4 + 0]) * mul, __uint_as_float(u[8 * v4 + 1]) * mul),
-                pack_bf16x2(__uint_as_float(u[8 * v4 + 2]) * mul, __uint_as_float(u[8 * v4 + 3]) * mul),
-                pack_bf16x2(__uint_as_float(u[8 * v4 + 4]) * mul, __uint_as_float(u[8 * v4 + 5]) * mul),
-                pack_bf16x2(__uint_as_float(u[8 * v4 + 6]) * mul, __uint_as_float(u[8 * v4 + 7]) * mul));
-        }
+        for (int v4 = 0; v4 < 4; ++v4)
+          *reinterpret_cast<uint4*>(stage + (c >> 1) * 4096 + sw128_offset(lane, (c & 1) * 4 + v4)) =
+              make_uint4(
+                  pack_bf16x2(__uint_as_float(u[8 * v4 + 0]) * mul, __uint_as_float(u[8 * v4 + 1]) * mul),
+                  pack_bf16x2(__uint_as_float(u[8 * v4 + 2]) * mul, __uint_as_float(u[8 * v4 + 3]) * mul),
+                  pack_bf16x2(__uint_as_float(u[8 * v4 + 4]) * mul, __uint_as_float(u[8 * v4 + 5]) * mul),
+                  pack_bf16x2(__uint_as_float(u[8 * v4 + 6]) * mul, __uint_as_float(u[8 * v4 + 7]) * mul));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      const int r0 = k0 + (warp & 3) * 32;
+      if (lane == 0 && r0 < N) {
+#pragma unroll
+        for (int ch = 0; ch < C::kChunks; ++ch)
+          tma_store_4d(half == 0 ? &tm_dk : &tm_dv, stage + ch * 4096, 64 * ch, h, r0, b);
+        bulk_commit();
+        bulk_wait_all();  // the stores have completed before the CTA's shared memory goes away
       }
     }
   } else if (wg == 2) {
@@ -416,6 +426,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       //   [ds_ready n] dQ_n = dS_n K (R2) ; dK += dS^T_n Q_n -> releases Q_n
       //   [dq_empty n] dP^T_{n+1} = V dO_{n+1}^T (R2)
       // so the next S^T and dV overlap the dS computation, and the dQ drain only gates dP.
+      // (Splitting dK in halves around dP^T_{n+1}, so that the compute warps get dP^T sooner,
+      // measured 10 % slower at N = 16k: the tensor pipe then idles while the drain warps
+      // empty the dQ columns, which all of dK used to cover.)
       if (lane == 0) {
         constexpr uint32_t id_sdp = idesc_bf16_f32(BM, BN, 0, 0);  // K_j Q_i^T, V_j dO_i^T
         constexpr uint32_t id_dkdv = idesc_bf16_f32(BM, D, 0, 1);  // P^T dO_i, dS^T Q_i
@@ -643,8 +656,7 @@ static cudaError_t launch_main_t(const BwdArgs& a, cudaStream_t st) {
   const int num_kvtiles = (a.N + BM - 1) / BM;
   const long long grid = static_cast<long long>(a.B) * a.H * num_kvtiles;
   kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, st>>>(
-      a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.lse2, a.delta, a.dq_acc,
-      static_cast<__nv_bfloat16*>(a.dk), static_cast<__nv_bfloat16*>(a.dv), a.B, a.H, a.N, n_pad,
+      a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.tm_dk, a.tm_dv, a.lse2, a.delta, a.dq_acc, a.B, a.H, a.N, n_pad,
       a.scale, a.scale * kLog2e, num_kvtiles, a.status, kDefaultWaitTimeoutNs);
   return cudaGetLastError();
 }

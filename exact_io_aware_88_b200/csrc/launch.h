@@ -29,6 +29,7 @@ struct FwdArgs {
 
 struct BwdArgs {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;  // 4-D maps, box {64,1,128,1}
+  CUtensorMap tm_dk, tm_dv;             // outputs, box {64,1,32,1} (one warp's rows)
   const void* o;
   const void* dO;
   const float* lse;
