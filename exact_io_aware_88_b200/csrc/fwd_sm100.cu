@@ -85,7 +85,7 @@ struct Cfg {
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
   static constexpr int kBarBytes = 512;              // Bars (size checked below)
-  // Block-sparse bitmasks: loader (2 tiles), MMA issuer (2), softmax warpgroup 0 and 1.
+  // Block-sparse bitmasks: loader, (unused), softmax warpgroups 0 and 1 (one copy per warp).
   static constexpr int kOffMask = kOffBar + kBarBytes;
   static constexpr int kMaskBytes = (2 + 2 + 8) * 32 * 4;  // + one copy per softmax warp
   // O epilogue: one staging box per softmax warp (32 rows x 128 bytes, 128-byte swizzled),
@@ -100,9 +100,12 @@ struct Cfg {
 
 struct Bars {
   uint64_t q_full, q_empty;
-  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+  uint64_t k_full[5], k_empty[5], v_full[4], v_empty[4];  // block-sparse: one more K stage
   uint64_t s_full[2], p_full[2], o_done[2], o_free[2];
   uint64_t p_half[2];  // P_t of the first 64 keys is in TMEM (and O_t rescaled)
+  // Block-sparse: softmax warpgroup 1 has published its row maximum and sum (merge_ready);
+  // warpgroup 0 has read them (merge_free).
+  uint64_t merge_ready, merge_free;
   // End-of-CTA protocol check: [0] K/V tiles loaded, [1] units loaded, [2] K/V tiles
   // consumed by the MMA lane, [3] its units, [4 + t] softmax t's steps, [6 + t] S products
   // issued for tile t, [8 + t] softmax t's units.
@@ -196,18 +199,25 @@ __global__ void pack_mask_kernel(const uint8_t* __restrict__ mask, uint32_t* __r
   words[i] = bits;
 }
 
-// Copies the pair's two tiles' words (tile 2*pair+t, zero for a tile past the last) into
-// this role's shared-memory copy: 2 x 128 bytes in 16-byte pieces.
-__device__ __forceinline__ void copy_pair_words(uint32_t* dst, const uint32_t* __restrict__ words,
-                                                int pair, int nq_tiles) {
+// Copies query tile qt's words into this role's shared-memory copy (128 bytes, 16 at a time).
+__device__ __forceinline__ void copy_tile_words(uint32_t* dst, const uint32_t* __restrict__ words,
+                                                int qt) {
+  const uint4* src = reinterpret_cast<const uint4*>(words + static_cast<size_t>(qt) * kMaskWords);
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int qt = 2 * pair + t;
-    const uint4* src = reinterpret_cast<const uint4*>(words + static_cast<size_t>(qt) * kMaskWords);
-    uint4* d4 = reinterpret_cast<uint4*>(dst + t * kMaskWords);
+  for (int i = 0; i < kMaskWords / 4; ++i) d4[i] = __ldg(src + i);
+}
+
+// Number of active key tiles of query tile qt (set bits of its words).
+__device__ __forceinline__ int count_tile_words(const uint32_t* __restrict__ words, int qt) {
+  const uint4* src = reinterpret_cast<const uint4*>(words + static_cast<size_t>(qt) * kMaskWords);
+  int n = 0;
 #pragma unroll
-    for (int i = 0; i < kMaskWords / 4; ++i) d4[i] = qt < nq_tiles ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+  for (int i = 0; i < kMaskWords / 4; ++i) {
+    const uint4 v = __ldg(src + i);
+    n += __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
   }
+  return n;
 }
 
 // Maximum of n values as a tree of 3-input max operations (depth log3 n).
@@ -231,9 +241,13 @@ __device__ __forceinline__ float tree_max(const float* v) {
 // F8: tm_q / tm_k map E4M3 [B][N][H][d], tm_v maps E4M3 V^T [B][H][d][Npad] (keys
 // contiguous), and scales[3][B*H] holds the per-head dequantisation scales of Q, K, V.
 // SPARSE: mask_words (pack_mask_kernel's output, kMaskWords words per query tile) selects the
-// 128 x 128 blocks worked on (block-sparse attention); the loader streams the union of the
-// pair's active key tiles, each softmax warpgroup walks its own, and a query tile with none
-// gets O = 0, LSE = -inf.
+// 128 x 128 blocks worked on (block-sparse attention).  A unit is then one query tile, not a
+// pair: Q is loaded once, the loader streams the tile's active key tiles in order, and they
+// go to the two ping-pong slots in turn (slot t takes the active key tiles k = t, t+2, ...),
+// each slot keeping its own running max, sum and O.  So both slots stay busy whatever the
+// mask, and at the end softmax warpgroup 0 merges the two partial results exactly, as the
+// split-KV merge does: O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) + l_1 2^(m_1-m)),
+// m = max(m_0, m_1).  A query tile with no active block gets O = 0, LSE = -inf.
 template <int D, bool CAUSAL, bool F8, bool SPARSE = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -242,6 +256,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                const uint32_t* __restrict__ mask_words, int B, int H, int N, float scale_log2,
                int num_pairs, int* status, uint64_t timeout_ns) {
   using C = Cfg<D, F8>;
+  constexpr int kKSt = SPARSE ? C::kStages + 1 : C::kStages;  // K ring depth
+  constexpr int kVSt = C::kStages;                            // V ring depth
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {  // 128-byte-swizzled tiles need a 1024-aligned base
     if (threadIdx.x == 0) atomicCAS(status, FA_OK, FA_ERR_UNSUPPORTED);
@@ -258,9 +274,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < kKSt; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < kVSt; ++s) {
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
@@ -271,6 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->o_done[t], 1);
       mbar_init(&bars->o_free[t], BM);
     }
+    mbar_init(&bars->merge_ready, BM);
+    mbar_init(&bars->merge_free, BM);
     mbar_init(&bars->drain, 1);
     bars->abort.flag = 0;
     fence_mbar_init();
@@ -285,7 +305,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = bars->tmem_base;
   Abort* ab = &bars->abort;
   uint8_t* sQ = smem + C::kOffQ;
-  uint8_t* sK = smem + C::kOffK;
+  // Block-sparse units hold one query tile, so Q1's slot becomes one more K stage (it sits
+  // right before the K ring): K runs kStages + 1 deep, V kStages.
+  uint8_t* sK = SPARSE ? smem + C::kOffQ + C::kTileBytes : smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
   const int wg = warp >> 2;
 
@@ -293,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (wg < 2) {
     regs_set<kRegsLaunch, kRegsSoftmax<F8>>();
     // ------------------------------------------------------------------ softmax warps
-    const int t = wg;                      // query tile of the pair
+    const int t = wg;                      // query tile of the pair (block-sparse: slot)
     const int r = (warp & 3) * 32 + lane;  // row within the tile == TMEM lane
     const uint32_t lane_base = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t colS = BN * t;
@@ -306,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (u >= num_units) break;
       const Unit x = decode_unit<CAUSAL>(u, BH, num_pairs);
       const int b = x.bh / H, h = x.bh % H;
-      const int q0 = (2 * x.pair + t) * BM;
+      const int q0 = (SPARSE ? x.pair : 2 * x.pair + t) * BM;
       const int row = q0 + r;
       const int nkv = kv_tiles<CAUSAL>(x.pair, t, kv_total);
       // Logit scale in log2 units (8-bit path: times the Q and K dequantisation scales) and
@@ -321,17 +343,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       PairMask pm;
       if constexpr (SPARSE) {
         uint32_t* words = reinterpret_cast<uint32_t*>(smem + C::kOffMask) + (4 + warp) * kMaskWords;
-        const int qt = 2 * x.pair + t;
         __syncwarp();  // every lane is done with the previous unit's words
-        words[lane] = qt < (N + BM - 1) / BM
-                          ? __ldg(mask_words + static_cast<size_t>(qt) * kMaskWords + lane)
-                          : 0u;
+        words[lane] = __ldg(mask_words + static_cast<size_t>(x.pair) * kMaskWords + lane);
         __syncwarp();
-        pm.w0 = pm.w1 = words;  // only tile t is asked for
+        pm.w0 = pm.w1 = words;
       }
+      // Block-sparse: this slot takes every other active key tile (slot 1 skips the first).
       BitIter it;
-      if constexpr (SPARSE) it.init(pm.w0);
-      for (int j = SPARSE ? it.pop() : 0; SPARSE ? j >= 0 : j < nkv; j = SPARSE ? it.pop() : j + 1) {
+      if constexpr (SPARSE) {
+        it.init(pm.w0);
+        if (t == 1) it.pop();
+      }
+      auto next_j = [&]() -> int {
+        const int jj = it.pop();
+        it.pop();  // the other slot's
+        return jj;
+      };
+      for (int j = SPARSE ? next_j() : 0; SPARSE ? j >= 0 : j < nkv; j = SPARSE ? next_j() : j + 1) {
         // Decisions guarding warp-collective tcgen05.ld/st are made warp-uniform.
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], ns & 1, ab, status, timeout_ns));
         if (!ok) break;
@@ -514,51 +542,108 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // -------------------------------------------------------------- epilogue
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[t], units & 1, ab, status, timeout_ns));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t o[D];
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c)
-        tmem_ld64(lane_base + colO + 64 * c, *reinterpret_cast<uint32_t(*)[64]>(&o[64 * c]));
-      tc_fence_before();
-      mbar_arrive(&bars->o_free[t]);  // the next unit's first PV may overwrite O_t now
-      ++units;
-      // A query tile with no active block (block-sparse) has l = 0 and O_t holds nothing of
-      // this unit: O = 0, LSE = -inf.
-      const bool empty = SPARSE && l == 0.f;
-      if (empty) {
-#pragma unroll
-        for (int i = 0; i < D; ++i) o[i] = 0u;
-      }
-      if (row < N)
-        lse[static_cast<size_t>(x.bh) * N + row] =
-            empty ? -INFINITY : (m + __log2f(l)) * 0.69314718055994531f;
       // O = O / l in bf16, written as whole 128-byte lines: each warp stages its 32 rows in
       // boxes of 64 head-dim elements (128-byte swizzle: conflict-free 16-byte shared stores)
       // and lane 0 hands each box to a TMA store, which clips the rows past N.  Before a box
       // is refilled, the store that read it must be done reading.
-      const float inv_l = empty ? 0.f : out_mul / l;
       const int r0 = q0 + (warp & 3) * 32;
       uint8_t* stage = smem + C::kOffStage + warp * C::kStageBytes;
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        if (lane == 0) bulk_wait_read_all();
-        __syncwarp();
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-          const uint32_t* e = &o[64 * c + 8 * p];
-          *reinterpret_cast<uint4*>(stage + sw128_offset(lane, p)) = make_uint4(
-              pack_bf16x2(__uint_as_float(e[0]) * inv_l, __uint_as_float(e[1]) * inv_l),
-              pack_bf16x2(__uint_as_float(e[2]) * inv_l, __uint_as_float(e[3]) * inv_l),
-              pack_bf16x2(__uint_as_float(e[4]) * inv_l, __uint_as_float(e[5]) * inv_l),
-              pack_bf16x2(__uint_as_float(e[6]) * inv_l, __uint_as_float(e[7]) * inv_l));
+      if constexpr (SPARSE) {
+        // The two slots' partial results of the one query tile.  Warpgroup 1 publishes its
+        // row maximum and sum in shared memory (its own staging boxes, which this mode does
+        // not use otherwise); warpgroup 0 merges both slots' O straight out of TMEM (the same
+        // lanes), writes O and the LSE, and then hands both O regions back.
+        float* mg = reinterpret_cast<float*>(smem + C::kOffStage + 4 * C::kStageBytes);
+        if (t == 1) {
+          if (units > 0) {  // warpgroup 0 has read the previous unit's values
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(&bars->merge_free, (units - 1) & 1, ab, status, timeout_ns));
+            if (!ok) break;
+          }
+          mg[r] = m;
+          mg[BM + r] = l;
+          mbar_arrive(&bars->merge_ready);
+          ++units;
+          continue;
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && r0 < N) {
-          tma_store_4d(&tm_o, stage, 64 * c, h, r0, b);
-          bulk_commit();
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[0], units & 1, ab, status, timeout_ns) &&
+                                         mbar_wait(&bars->o_done[1], units & 1, ab, status, timeout_ns) &&
+                                         mbar_wait(&bars->merge_ready, units & 1, ab, status, timeout_ns));
+        if (!ok) break;
+        tc_fence_after();
+        const float m1 = mg[r], l1 = mg[BM + r];
+        mbar_arrive(&bars->merge_free);
+        // A slot that saw no key tile has l = 0 (and m = -inf): it contributes nothing.
+        const float mm = fmaxf(m, m1);
+        const float f0 = l > 0.f ? ex2_approx(m - mm) : 0.f;
+        const float f1 = l1 > 0.f ? ex2_approx(m1 - mm) : 0.f;
+        const float lt = l * f0 + l1 * f1;
+        const bool empty = !(lt > 0.f);
+        const float a0 = empty ? 0.f : f0 / lt, a1 = empty ? 0.f : f1 / lt;
+        if (row < N)
+          lse[static_cast<size_t>(x.bh) * N + row] =
+              empty ? -INFINITY : (mm + __log2f(lt)) * 0.69314718055994531f;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t o0[64], o1[64];
+          tmem_ld64(lane_base + C::kColO + 64 * c, o0);
+          tmem_ld64(lane_base + C::kColO + 128 + 64 * c, o1);
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+#pragma unroll
+          for (int p = 0; p < 8; ++p) {
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              v[i] = __uint_as_float(o0[8 * p + i]) * a0 + __uint_as_float(o1[8 * p + i]) * a1;
+            *reinterpret_cast<uint4*>(stage + sw128_offset(lane, p)) =
+                make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                           pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && r0 < N) {
+            tma_store_4d(&tm_o, stage, 64 * c, h, r0, b);
+            bulk_commit();
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->o_free[0]);  // the next unit's first PVs may overwrite O_0, O_1
+        mbar_arrive(&bars->o_free[1]);
+        ++units;
+      } else {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[t], units & 1, ab, status, timeout_ns));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t o[D];
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tmem_ld64(lane_base + colO + 64 * c, *reinterpret_cast<uint32_t(*)[64]>(&o[64 * c]));
+        tc_fence_before();
+        mbar_arrive(&bars->o_free[t]);  // the next unit's first PV may overwrite O_t now
+        ++units;
+        if (row < N)
+          lse[static_cast<size_t>(x.bh) * N + row] = (m + __log2f(l)) * 0.69314718055994531f;
+        const float inv_l = out_mul / l;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+#pragma unroll
+          for (int p = 0; p < 8; ++p) {
+            const uint32_t* e = &o[64 * c + 8 * p];
+            *reinterpret_cast<uint4*>(stage + sw128_offset(lane, p)) = make_uint4(
+                pack_bf16x2(__uint_as_float(e[0]) * inv_l, __uint_as_float(e[1]) * inv_l),
+                pack_bf16x2(__uint_as_float(e[2]) * inv_l, __uint_as_float(e[3]) * inv_l),
+                pack_bf16x2(__uint_as_float(e[4]) * inv_l, __uint_as_float(e[5]) * inv_l),
+                pack_bf16x2(__uint_as_float(e[6]) * inv_l, __uint_as_float(e[7]) * inv_l));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && r0 < N) {
+            tma_store_4d(&tm_o, stage, 64 * c, h, r0, b);
+            bulk_commit();
+          }
         }
       }
     }
@@ -589,78 +674,62 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (units > 0 &&
               !(ok = mbar_wait(&bars->q_empty, (units - 1) & 1, ab, status, timeout_ns)))
             break;
-          mbar_arrive_expect_tx(&bars->q_full, 2 * C::kTileBytes);
-          for (int t = 0; t < 2; ++t)
+          // Dense: the pair's two query tiles.  Block-sparse: the unit's one query tile (both
+          // slots read it).
+          constexpr int kQTiles = SPARSE ? 1 : 2;
+          mbar_arrive_expect_tx(&bars->q_full, kQTiles * C::kTileBytes);
+          for (int t = 0; t < kQTiles; ++t)
             for (int c = 0; c < C::kChunks; ++c)
               tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &tm_q, &bars->q_full,
-                          c * C::kChunkElems, h, (2 * x.pair + t) * BM, b, pol_q);
+                          c * C::kChunkElems, h, (SPARSE ? x.pair : 2 * x.pair + t) * BM, b, pol_q);
           ++units;
           const int nkv = kv_tiles<CAUSAL>(x.pair, 1, kv_total);
-          PairMask pm;
+          // Block-sparse: the query tile's active key tiles, in order.
+          BitIter it0;
           if constexpr (SPARSE) {
             uint32_t* words = reinterpret_cast<uint32_t*>(smem + C::kOffMask);
-            copy_pair_words(words, mask_words, x.pair, (N + BM - 1) / BM);
-            pm.w0 = words;
-            pm.w1 = words + kMaskWords;
+            copy_tile_words(words, mask_words, x.pair);
+            it0.init(words);
           }
-          BitIter it0, it1;
-          int h0 = -1, h1 = -1;  // next active key tile of each tile (sparse)
-          if constexpr (SPARSE) {
-            it0.init(pm.w0);
-            it1.init(pm.w1);
-            h0 = it0.pop();
-            h1 = it1.pop();
-          }
-          // Union order: the smaller head; a head equal to it advances.
-          auto union_pop = [&]() -> int {
-            const int jj = h0 < 0 ? h1 : (h1 < 0 ? h0 : min(h0, h1));
-            if (jj >= 0) {
-              if (h0 == jj) h0 = it0.pop();
-              if (h1 == jj) h1 = it1.pop();
-            }
-            return jj;
-          };
-          for (int j = SPARSE ? union_pop() : 0; SPARSE ? j >= 0 : j < nkv;
-               j = SPARSE ? union_pop() : j + 1, ++g) {
-            const int s = g % C::kStages;
-            const uint32_t ph = ((g / C::kStages) - 1) & 1;
-            if (g >= C::kStages &&
-                !(ok = mbar_wait(&bars->k_empty[s], ph, ab, status, timeout_ns)))
+          for (int j = SPARSE ? it0.pop() : 0; SPARSE ? j >= 0 : j < nkv;
+               j = SPARSE ? it0.pop() : j + 1, ++g) {
+            const int s = g % kKSt, sv = g % kVSt;
+            if (g >= kKSt &&
+                !(ok = mbar_wait(&bars->k_empty[s], ((g / kKSt) - 1) & 1, ab, status, timeout_ns)))
               break;
             mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes);
             for (int c = 0; c < C::kChunks; ++c)
               tma_load_4d(sK + s * C::kTileBytes + c * C::kChunkBytes, &tm_k, &bars->k_full[s],
                           c * C::kChunkElems, h, j * BN, b, pol_kv);
-            if (g >= C::kStages &&
-                !(ok = mbar_wait(&bars->v_empty[s], ph, ab, status, timeout_ns))) {
+            if (g >= kVSt &&
+                !(ok = mbar_wait(&bars->v_empty[sv], ((g / kVSt) - 1) & 1, ab, status, timeout_ns))) {
               ++g;  // K of this tile is in flight: count it for the drain below
               break;
             }
-            mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
+            mbar_arrive_expect_tx(&bars->v_full[sv], C::kTileBytes);
             if constexpr (F8) {  // V^T box: 128 keys x 128 head-dim rows
-              tma_load_4d(sV + s * C::kTileBytes, &tm_v, &bars->v_full[s], j * BN, 0, h, b,
+              tma_load_4d(sV + sv * C::kTileBytes, &tm_v, &bars->v_full[sv], j * BN, 0, h, b,
                           pol_kv);
             } else {
               for (int c = 0; c < C::kChunks; ++c)
-                tma_load_4d(sV + s * C::kTileBytes + c * C::kChunkBytes, &tm_v, &bars->v_full[s],
+                tma_load_4d(sV + sv * C::kTileBytes + c * C::kChunkBytes, &tm_v, &bars->v_full[sv],
                             c * 64, h, j * BN, b, pol_kv);
             }
           }
         }
         // Drain: no copy into shared memory may still be in flight when the CTA exits.
-        // Only the last Q pair and the last kStages K/V tiles can be outstanding.  (On the
-        // abort path a V copy may not have been issued; its wait then runs out harmlessly.)
+        // Only the last Q tiles, the last kKSt K tiles and the last kVSt V tiles can be
+        // outstanding.  (On the abort path the last V copy may not have been issued; its wait
+        // then runs out harmlessly.)
         bars->count[0] = g;
         bars->count[1] = units;
         Abort local{0};
         if (units > 0) mbar_wait(&bars->q_full, (units - 1) & 1, &local, status, timeout_ns);
-        for (int gg = max(0, g - C::kStages); gg < g; ++gg) {
-          mbar_wait(&bars->k_full[gg % C::kStages], (gg / C::kStages) & 1, &local, status,
-                    timeout_ns);
+        for (int gg = max(0, g - kKSt); gg < g; ++gg)
+          mbar_wait(&bars->k_full[gg % kKSt], (gg / kKSt) & 1, &local, status, timeout_ns);
+        for (int gg = max(0, g - kVSt); gg < g; ++gg)
           if (ok || gg < g - 1)
-            mbar_wait(&bars->v_full[gg % C::kStages], (gg / C::kStages) & 1, &local, status,
-                      timeout_ns);
-        }
+            mbar_wait(&bars->v_full[gg % kVSt], (gg / kVSt) & 1, &local, status, timeout_ns);
       }
     } else if (warp == kWarpMma) {
       // ---------------------------------------------------------------- MMA issuer
@@ -677,7 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto issue_s = [&](int t, int s) {  // S_t = Q_t K^T (both K-major over the head dim)
           (t ? s_issued1 : s_issued0) += 1;
           const uint32_t kb = aK + s * C::kTileBytes;
-          const uint32_t qb = aQ + t * C::kTileBytes;
+          const uint32_t qb = aQ + (SPARSE ? 0 : t * C::kTileBytes);  // sparse: one Q, both slots
           // One MMA per 32 bytes of the head dim (16 bf16 or 32 E4M3 elements).
 #pragma unroll
           for (int kk = 0; kk < C::kRowBytes / 32; ++kk) {
@@ -733,158 +802,60 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         if constexpr (SPARSE) {
-          // Block-sparse issue order.  Key tiles come in the union order of the two query
-          // tiles' active lists (the loader's ring order).  At each such key tile j: first
-          // any S_t(j) still owed (deferred because j was not the next ring tile when
-          // PV_t(previous) was issued), then for every tile active at j: PV_t(j) followed,
-          // when t's next active tile is also the next ring tile, by S_t(next) at once (the
-          // dense order).  A K stage is released once every S on it has been issued.
-          const int nq_tiles = (N + BM - 1) / BM;
+          // Block-sparse issue order.  The unit's cnt active key tiles sit at ring positions
+          // g .. g+cnt-1 in order; the k-th goes to slot k % 2.  After S_0(k=0) and S_1(k=1),
+          // for k = 0, 1, 2, ...: PV_{k%2}(k), then that slot's next S (k+2) at once, so the
+          // order is the dense one, PV_0, S_0, PV_1, S_1, with the two slots on different key
+          // tiles.  Each K stage is read by one S and each V stage by one PV, so each is
+          // released right after it.
           for (int r = 0; ok; ++r) {
             const int u = unit_of_round(r, G);
             if (u >= num_units) break;
             const Unit x = decode_unit<CAUSAL>(u, BH, num_pairs);
-            PairMask pm;
-            {
-              uint32_t* words = reinterpret_cast<uint32_t*>(smem + C::kOffMask) + 2 * kMaskWords;
-              copy_pair_words(words, mask_words, x.pair, nq_tiles);
-              pm.w0 = words;
-              pm.w1 = words + kMaskWords;
-            }
+            const int cnt = count_tile_words(mask_words, x.pair);
             if (!(ok = mbar_wait(&bars->q_full, units & 1, ab, status, timeout_ns))) break;
-            // Per-tile state, kept in scalars (t is a compile-time constant below).  For each
-            // tile: cur_t = its next key tile, nx_t = the one after, nx2_t = the one after
-            // that (from a bit iterator over its mask words).
-            BitIter it0, it1;
-            it0.init(pm.w0);
-            it1.init(pm.w1);
-            int cur0 = it0.pop(), cur1 = it1.pop();
-            int nx0 = cur0 < 0 ? -1 : it0.pop(), nx1 = cur1 < 0 ? -1 : it1.pop();
-            int nx20 = nx0 < 0 ? -1 : it0.pop(), nx21 = nx1 < 0 ? -1 : it1.pop();
-            bool sd0 = false, sd1 = false;                      // S_t(cur_t) issued
-            bool fp0 = true, fp1 = true;                        // first PV of the unit
-            bool ls0 = cur0 < 0, ls1 = cur1 < 0;                // no S left to issue for t
-            bool q_released = false;
-            auto release_q = [&]() {
-              if (!q_released && ls0 && ls1) {
-                umma_commit(&bars->q_empty);
-                q_released = true;
-              }
-            };
-            // A tile with no active key tile has nothing to accumulate: its O is signalled done
-            // at once, but only after its softmax warpgroup has read the previous unit's O.
-            // Without that wait o_done could complete twice (the previous unit's last PV and
-            // this commit track the same products) before the warpgroup polls it, and a wait
-            // on a phase's parity cannot tell two completions from none.
-            if (cur0 < 0) {
+            // A slot with no key tile has nothing to accumulate: its O is signalled done at
+            // once, but only after warpgroup 0 has read the previous unit's O (without that
+            // wait o_done could complete twice before it is polled, and a wait on a phase's
+            // parity cannot tell two completions from none).
+            for (int t = 0; t < 2 && ok; ++t) {
+              if (cnt > t) continue;
               if (units > 0 &&
-                  !(ok = mbar_wait(&bars->o_free[0], (units - 1) & 1, ab, status, timeout_ns)))
+                  !(ok = mbar_wait(&bars->o_free[t], (units - 1) & 1, ab, status, timeout_ns)))
                 break;
-              umma_commit(&bars->o_done[0]);
+              umma_commit(&bars->o_done[t]);
             }
-            if (cur1 < 0) {
-              if (units > 0 &&
-                  !(ok = mbar_wait(&bars->o_free[1], (units - 1) & 1, ab, status, timeout_ns)))
-                break;
-              umma_commit(&bars->o_done[1]);
-            }
-            int j = cur0 < 0 ? cur1 : (cur1 < 0 ? cur0 : min(cur0, cur1));
-            int gu = g;  // ring position of key tile j
-            if (j >= 0) {
-              const int s = gu % C::kStages;
-              if (!(ok = mbar_wait(&bars->k_full[s], (gu / C::kStages) & 1, ab, status,
-                                   timeout_ns)))
-                break;
+            if (!ok) break;
+            if (cnt == 0) umma_commit(&bars->q_empty);
+            auto issue_s_at = [&](int k) -> bool {  // S_{k%2} on ring position g + k
+              const int pos = g + k, s = pos % kKSt;
+              if (!mbar_wait(&bars->k_full[s], (pos / kKSt) & 1, ab, status, timeout_ns))
+                return false;
               tc_fence_after();
-              if (cur0 == j) {
-                issue_s(0, s);
-                sd0 = true;
-                ls0 = nx0 < 0;
-              }
-              if (cur1 == j) {
-                issue_s(1, s);
-                sd1 = true;
-                ls1 = nx1 < 0;
-              }
-              umma_commit(&bars->k_empty[s]);  // every tile active at j is served
-            }
-            release_q();
-            while (ok && j >= 0) {
-              const int s = gu % C::kStages;
-              const int sn = (gu + 1) % C::kStages;
-              // Everything this step needs from the masks, before any wait.
-              const bool on0 = cur0 == j, on1 = cur1 == j;
-              const int nt0 = on0 ? nx0 : cur0;
-              const int nt1 = on1 ? nx1 : cur1;
-              const int jn = (nt0 < 0) ? nt1 : ((nt1 < 0) ? nt0 : min(nt0, nt1));
-              const bool last0 = nt0 < 0 || (on0 ? nx20 : nx0) < 0;
-              const bool last1 = nt1 < 0 || (on1 ? nx21 : nx1) < 0;
-              // S owed on j (its K stage is still held for it).
-              const bool owe0 = on0 && !sd0, owe1 = on1 && !sd1;
-              if (owe0 || owe1) {
-                tc_fence_after();
-                if (owe0) {
-                  issue_s(0, s);
-                  ls0 = !(nt0 >= 0);
-                }
-                if (owe1) {
-                  issue_s(1, s);
-                  ls1 = !(nt1 >= 0);
-                }
-                umma_commit(&bars->k_empty[s]);
-                release_q();
-              }
-              if (!(ok = mbar_wait(&bars->v_full[s], (gu / C::kStages) & 1, ab, status,
+              issue_s(k & 1, s);
+              umma_commit(&bars->k_empty[s]);
+              if (k == cnt - 1) umma_commit(&bars->q_empty);  // the unit's last S product
+              return true;
+            };
+            if (cnt >= 1 && !(ok = issue_s_at(0))) break;
+            if (cnt >= 2 && !(ok = issue_s_at(1))) break;
+            for (int k = 0; ok && k < cnt; ++k) {
+              const int t = k & 1, pos = g + k, s = pos % kVSt;
+              if (!(ok = mbar_wait(&bars->v_full[s], (pos / kVSt) & 1, ab, status,
                                    timeout_ns)))
                 break;
-              if (jn >= 0 && !(ok = mbar_wait(&bars->k_full[sn], ((gu + 1) / C::kStages) & 1, ab,
-                                               status, timeout_ns)))
+              if (k < 2 && units > 0 &&
+                  !(ok = mbar_wait(&bars->o_free[t], (units - 1) & 1, ab, status, timeout_ns)))
                 break;
-              // The V stage is released right after the last PV that reads it, before that
-              // tile's next S, so that its reload is not held up by the S product.
-              auto pv_then_next_s = [&](auto tc, bool on, bool& fp, int& cur, bool& sd, bool& ls,
-                                        int nt, bool last, bool last_pv) -> bool {
-                constexpr int t = decltype(tc)::value;
-                if (!on) return true;
-                if (fp && units > 0 &&
-                    !mbar_wait(&bars->o_free[t], (units - 1) & 1, ab, status, timeout_ns))
-                  return false;
-                if (!issue_pv(t, s, fp, np[t])) return false;
-                if (last_pv) umma_commit(&bars->v_empty[s]);
-                fp = false;
-                cur = nt;
-                sd = false;
-                if (nt < 0) {
-                  umma_commit(&bars->o_done[t]);
-                } else if (nt == jn) {
-                  issue_s(t, sn);
-                  sd = true;
-                  ls = last;
-                }
-                return true;
-              };
-              if (!(ok = pv_then_next_s(std::integral_constant<int, 0>{}, on0, fp0, cur0, sd0, ls0,
-                                        nt0, last0, !on1)))
-                break;
-              if (!(ok = pv_then_next_s(std::integral_constant<int, 1>{}, on1, fp1, cur1, sd1, ls1,
-                                        nt1, last1, true)))
-                break;
-              // Advance the lookahead of the tiles that moved on.
-              if (on0) {
-                nx0 = nx20;
-                nx20 = nx20 < 0 ? -1 : it0.pop();
+              if (!(ok = issue_pv(t, s, k < 2, np[t]))) break;
+              umma_commit(&bars->v_empty[s]);
+              if (k + 2 < cnt) {
+                if (!(ok = issue_s_at(k + 2))) break;
+              } else {
+                umma_commit(&bars->o_done[t]);  // slot t's last PV of the unit
               }
-              if (on1) {
-                nx1 = nx21;
-                nx21 = nx21 < 0 ? -1 : it1.pop();
-              }
-              if (jn >= 0 && !((cur0 == jn && !sd0) || (cur1 == jn && !sd1)))
-                umma_commit(&bars->k_empty[sn]);  // no S owed on jn: its K stage is free
-              release_q();
-              j = jn;
-              ++gu;
             }
-            g = gu;
+            g += cnt;
             ++units;
           }
         } else {
@@ -1004,7 +975,8 @@ static cudaError_t launch_t(const FwdArgs& a, cudaStream_t st) {
   if (fa_attr.numRegs != static_cast<int>(kRegsLaunch)) return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int num_pairs = (a.N + 2 * BM - 1) / (2 * BM);
+  // Units per (batch, head): pairs of query tiles (dense), single query tiles (block-sparse).
+  const int num_pairs = SPARSE ? (a.N + BM - 1) / BM : (a.N + 2 * BM - 1) / (2 * BM);
   const long long units = static_cast<long long>(a.B) * a.H * num_pairs;
   if (units > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const int grid = static_cast<int>(std::min<long long>(units, a.num_sms));

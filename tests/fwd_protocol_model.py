@@ -1,7 +1,9 @@
 """Discrete-event model of the forward kernel's barrier protocol (csrc/fwd_sm100.cu): one
 persistent CTA working through several units, its TMA producer, MMA issuer (dense and
 block-sparse issue orders) and two softmax warpgroups, the in-order tensor pipe with its
-commits, and TMA loads that land in any order.
+commits, and TMA loads that land in any order.  In the block-sparse mode a unit is one query
+tile whose active key tiles alternate between the two slots, and warpgroup 0 merges both
+slots' results (merge_ready / merge_free with warpgroup 1, o_done and o_free of both slots).
 
 Waits have the hardware's semantics: a wait for phase k of an mbarrier returns when the
 current phase's parity differs from k's, so a barrier that completes two phases before a
@@ -48,6 +50,8 @@ class Sim:
         self.p_half_pub = [0, 0]
         self.s_issued = [0, 0]
         self.o_read_units = [0, 0]   # epilogues done per tile
+        self.merge_pub = 0           # block-sparse: units whose slot-1 values are published
+        self.merge_read = 0          # ... and read by warpgroup 0
         self.o_unit_pv = [{}, {}]    # unit -> PVs executed
 
     def completed(self, bar):
@@ -66,14 +70,18 @@ class Sim:
 
 def run(mode, masks0, masks1, nkv_list, seed, stages=4, empty_tile_waits_o_free=True,
         split_p=False, max_steps=200000):
-    """mode 'dense' (nkv_list: (nkv0, nkv1) per unit) or 'sparse' (masks0 / masks1: the two
-    query tiles' sorted active key tiles per unit).  `stages` is the K/V ring depth (2 at
-    head dim 128, 4 at 64).  `empty_tile_waits_o_free=False` restores the earlier block-
-    sparse issue logic, which signalled an empty tile's O without waiting for o_free.
+    """mode 'dense' (nkv_list: (nkv0, nkv1) per unit) or 'sparse' (masks0: the unit's query
+    tile's sorted active key tiles, per unit; masks1 unused).  `stages` is the K/V ring depth
+    (2 at head dim 128, 4 at 64).  `empty_tile_waits_o_free=False` signals an empty slot's O
+    without waiting for o_free (the race the kernel avoids).
     `split_p` (dense only): P is published in two halves (p_half, then p_full) and each half
     of PV is issued after its half, as on the 8-bit path.
     Returns "ok" or raises Deadlock / Hazard."""
     S_STAGES = stages
+    # Block-sparse units hold one query tile, and the kernel turns the second Q slot into one
+    # more K stage: K runs stages + 1 deep, V stages deep.
+    KS = stages + 1 if mode == "sparse" else stages
+    VS = stages
     rng = random.Random(seed)
     sim = Sim(rng)
     units = len(nkv_list) if mode == "dense" else len(masks0)
@@ -82,7 +90,8 @@ def run(mode, masks0, masks1, nkv_list, seed, stages=4, empty_tile_waits_o_free=
         if mode == "dense":
             n0, n1 = nkv_list[u]
             return list(range(n0)), list(range(n1))
-        return masks0[u], masks1[u]
+        lst = list(masks0[u])
+        return lst[0::2], lst[1::2]   # the slots' key tiles
 
     # ------------------------------------------------------------------ roles
     def loader():
@@ -94,19 +103,21 @@ def run(mode, masks0, masks1, nkv_list, seed, stages=4, empty_tile_waits_o_free=
                 raise Hazard("Q overwritten while S products still read it")
             sim.tma.append(("q_full", "Q", u))
             l0, l1 = tile_lists(u)
-            for j in sorted(set(l0) | set(l1)):
-                s = g % S_STAGES
-                if g >= S_STAGES:
-                    yield ("wait", f"k_empty{s}", g // S_STAGES - 1)
-                old = g - S_STAGES
+            for j in (sorted(set(l0) | set(l1)) if mode == "dense" else masks0[u]):
+                s = g % KS
+                if g >= KS:
+                    yield ("wait", f"k_empty{s}", g // KS - 1)
+                old = g - KS
                 if old >= 0 and sim.k_reads_pending.get(old, 0):
                     raise Hazard(f"K slot {s} reloaded while pos {old} still read")
                 sim.tma.append((f"k_full{s}", "K", g))
-                if g >= S_STAGES:
-                    yield ("wait", f"v_empty{s}", g // S_STAGES - 1)
+                sv = g % VS
+                if g >= VS:
+                    yield ("wait", f"v_empty{sv}", g // VS - 1)
+                old = g - VS
                 if old >= 0 and sim.v_reads_pending.get(old, 0):
-                    raise Hazard(f"V slot {s} reloaded while pos {old} still read")
-                sim.tma.append((f"v_full{s}", "V", g))
+                    raise Hazard(f"V slot {sv} reloaded while pos {old} still read")
+                sim.tma.append((f"v_full{sv}", "V", g))
                 g += 1
 
     def issue_s(t, pos, u):
@@ -195,91 +206,44 @@ def run(mode, masks0, masks1, nkv_list, seed, stages=4, empty_tile_waits_o_free=
         g = 0
         np_ = [0, 0]
         for u in range(units):
-            l0, l1 = list(masks0[u]), list(masks1[u])
-            it = [iter(l0), iter(l1)]
-
-            def pop(t):
-                return next(it[t], -1)
+            cnt = len(masks0[u])
             yield ("wait", "q_full", u)
-            cur = [pop(0), pop(1)]
-            nx = [pop(0) if cur[0] >= 0 else -1, pop(1) if cur[1] >= 0 else -1]
-            nx2 = [pop(0) if nx[0] >= 0 else -1, pop(1) if nx[1] >= 0 else -1]
-            sd = [False, False]
-            fp = [True, True]
-            ls = [cur[0] < 0, cur[1] < 0]
-            qrel = [False]
-
-            def release_q():
-                if not qrel[0] and ls[0] and ls[1]:
-                    commit("q_empty")
-                    qrel[0] = True
             for t in (0, 1):
-                if cur[t] < 0:
+                if cnt <= t:
                     if empty_tile_waits_o_free and u > 0:
                         yield ("wait", f"o_free{t}", u - 1)
                     commit(f"o_done{t}")
-            cands = [c for c in cur if c >= 0]
-            j = min(cands) if cands else -1
-            gu = g
-            if j >= 0:
-                s = gu % S_STAGES
-                yield ("wait", f"k_full{s}", gu // S_STAGES)
-                for t in (0, 1):
-                    if cur[t] == j:
-                        issue_s(t, gu, u)
-                        sd[t] = True
-                        ls[t] = nx[t] < 0
+            if cnt == 0:
+                commit("q_empty")
+
+            def issue_s_at(k):
+                pos = g + k
+                s = pos % KS
+                yield ("wait", f"k_full{s}", pos // KS)
+                issue_s(k & 1, pos, u)
                 commit(f"k_empty{s}")
-            release_q()
-            while j >= 0:
-                s = gu % S_STAGES
-                sn = (gu + 1) % S_STAGES
-                on = [cur[0] == j, cur[1] == j]
-                nt = [nx[t] if on[t] else cur[t] for t in (0, 1)]
-                c2 = [x for x in nt if x >= 0]
-                jn = min(c2) if c2 else -1
-                last = [nt[t] < 0 or (nx2[t] if on[t] else nx[t]) < 0 for t in (0, 1)]
-                owe = [on[t] and not sd[t] for t in (0, 1)]
-                if owe[0] or owe[1]:
-                    for t in (0, 1):
-                        if owe[t]:
-                            issue_s(t, gu, u)
-                            ls[t] = not (nt[t] >= 0)
-                    commit(f"k_empty{s}")
-                    release_q()
-                yield ("wait", f"v_full{s}", gu // S_STAGES)
-                if jn >= 0:
-                    yield ("wait", f"k_full{sn}", (gu + 1) // S_STAGES)
-                for t in (0, 1):
-                    if not on[t]:
-                        continue
-                    last_pv = (not on[1]) if t == 0 else True
-                    if fp[t] and u > 0:
-                        yield ("wait", f"o_free{t}", u - 1)
-                    yield ("wait", f"p_full{t}", np_[t])
-                    issue_pv(t, gu, u, fp[t])
-                    np_[t] += 1
-                    if last_pv:
-                        commit(f"v_empty{s}")
-                    fp[t] = False
-                    cur[t] = nt[t]
-                    sd[t] = False
-                    if nt[t] < 0:
-                        commit(f"o_done{t}")
-                    elif nt[t] == jn:
-                        issue_s(t, gu + 1, u)
-                        sd[t] = True
-                        ls[t] = last[t]
-                for t in (0, 1):
-                    if on[t]:
-                        nx[t] = nx2[t]
-                        nx2[t] = pop(t) if nx2[t] >= 0 else -1
-                if jn >= 0 and not ((cur[0] == jn and not sd[0]) or (cur[1] == jn and not sd[1])):
-                    commit(f"k_empty{sn}")
-                release_q()
-                j = jn
-                gu += 1
-            g = gu
+                if k == cnt - 1:
+                    commit("q_empty")
+            if cnt >= 1:
+                yield from issue_s_at(0)
+            if cnt >= 2:
+                yield from issue_s_at(1)
+            for k in range(cnt):
+                t = k & 1
+                pos = g + k
+                s = pos % VS
+                yield ("wait", f"v_full{s}", pos // VS)
+                if k < 2 and u > 0:
+                    yield ("wait", f"o_free{t}", u - 1)
+                yield ("wait", f"p_full{t}", np_[t])
+                issue_pv(t, pos, u, k < 2)
+                np_[t] += 1
+                commit(f"v_empty{s}")
+                if k + 2 < cnt:
+                    yield from issue_s_at(k + 2)
+                else:
+                    commit(f"o_done{t}")
+            g += cnt
 
     def softmax(t):
         ns = 0
@@ -300,11 +264,36 @@ def run(mode, masks0, masks1, nkv_list, seed, stages=4, empty_tile_waits_o_free=
                     yield ("step",)
                 sim.p_pub[t] += 1
                 sim.complete(f"p_full{t}")
-            yield ("wait", f"o_done{t}", u)
-            if sim.o_unit_pv[t].get(u, 0) != len(lst):
-                raise Hazard(f"softmax{t} read O of unit {u} before its PVs finished")
-            sim.o_read_units[t] += 1
-            sim.complete(f"o_free{t}")
+            if mode == "dense":
+                yield ("wait", f"o_done{t}", u)
+                if sim.o_unit_pv[t].get(u, 0) != len(lst):
+                    raise Hazard(f"softmax{t} read O of unit {u} before its PVs finished")
+                sim.o_read_units[t] += 1
+                sim.complete(f"o_free{t}")
+            elif t == 1:
+                # publish this slot's max and sum for the merge
+                if u > 0:
+                    yield ("wait", "merge_free", u - 1)
+                if sim.merge_read < u:
+                    raise Hazard(f"warpgroup 1 overwrote the merge values of unit {u - 1} unread")
+                sim.merge_pub = u + 1
+                sim.complete("merge_ready")
+            else:
+                # warpgroup 0 merges both slots' O and hands both back
+                lists = tile_lists(u)
+                yield ("wait", "o_done0", u)
+                yield ("wait", "o_done1", u)
+                yield ("wait", "merge_ready", u)
+                for tt in (0, 1):
+                    if sim.o_unit_pv[tt].get(u, 0) != len(lists[tt]):
+                        raise Hazard(f"merge read O{tt} of unit {u} before its PVs finished")
+                if sim.merge_pub < u + 1:
+                    raise Hazard(f"merge read warpgroup 1's values of unit {u} unpublished")
+                sim.merge_read = u + 1
+                sim.complete("merge_free")
+                for tt in (0, 1):
+                    sim.o_read_units[tt] += 1
+                    sim.complete(f"o_free{tt}")
 
     # ------------------------------------------------------------------ scheduler
     roles = {"load": loader(), "mma": mma_dense() if mode == "dense" else mma_sparse(),
@@ -372,14 +361,10 @@ def run(mode, masks0, masks1, nkv_list, seed, stages=4, empty_tile_waits_o_free=
 
 
 def random_masks(rng, units, nt, causal, density):
-    m0, m1 = [], []
+    """Block-sparse units: per unit, one query tile's sorted active key tiles."""
+    out = []
     for u in range(units):
-        p = rng.randrange(max(1, (nt + 1) // 2))
-        lists = []
-        for t in (0, 1):
-            qt = 2 * p + t
-            vis = range(nt) if not causal else range(min(nt, qt + 1))
-            lists.append(sorted(j for j in vis if qt < nt and rng.random() < density))
-        m0.append(lists[0])
-        m1.append(lists[1])
-    return m0, m1
+        qt = rng.randrange(max(1, nt))
+        vis = range(nt) if not causal else range(min(nt, qt + 1))
+        out.append(sorted(j for j in vis if rng.random() < density))
+    return out

@@ -12,17 +12,7 @@ from tests import fwd_protocol_model as model
 
 
 def _random_masks(rng, units, nt, causal, density):
-    m0, m1 = [], []
-    for _ in range(units):
-        p = rng.randrange(max(1, (nt + 1) // 2))
-        lists = []
-        for t in (0, 1):
-            qt = 2 * p + t
-            vis = range(nt) if not causal else range(min(nt, qt + 1))
-            lists.append(sorted(j for j in vis if qt < nt and rng.random() < density))
-        m0.append(lists[0])
-        m1.append(lists[1])
-    return m0, m1
+    return model.random_masks(rng, units, nt, causal, density)
 
 
 @pytest.mark.parametrize("stages,split_p", [(2, False), (4, False), (4, True)])
@@ -44,23 +34,50 @@ def test_dense_issue_order_is_safe(stages, split_p):
 def test_block_sparse_issue_order_is_safe(stages):
     rng = random.Random(10 + stages)
     for case in range(600):
-        m0, m1 = _random_masks(rng, rng.randrange(1, 5), rng.randrange(1, 12),
-                               rng.random() < 0.5, rng.choice([0.0, 0.2, 0.5, 0.9, 1.0]))
+        m0 = _random_masks(rng, rng.randrange(1, 5), rng.randrange(1, 12),
+                           rng.random() < 0.5, rng.choice([0.0, 0.2, 0.5, 0.9, 1.0]))
         for sched in range(4):
-            assert model.run("sparse", m0, m1, None, seed=100 * case + sched,
+            assert model.run("sparse", m0, None, None, seed=100 * case + sched,
                              stages=stages) == "ok"
 
 
 def test_model_sees_the_empty_tile_race():
-    """Unit 0: both query tiles have work; unit 1: both are empty.  With the earlier logic
-    the second unit's o_done commits can land before the softmax warpgroups poll the
-    first, which some schedule must expose."""
-    m0, m1 = [[0], []], [[0, 1], []]
+    """Unit 0: both slots have work; unit 1: the query tile has no active key tile.  If an
+    empty slot's o_done were committed without waiting for o_free, the second unit's commits
+    could land before warpgroup 0 polls the first, which some schedule must expose."""
+    m0 = [[0, 1], []]
     failures = 0
     for seed in range(40):
         try:
-            model.run("sparse", m0, m1, None, seed=seed, empty_tile_waits_o_free=False)
+            model.run("sparse", m0, None, None, seed=seed, empty_tile_waits_o_free=False)
         except (model.Deadlock, model.Hazard):
             failures += 1
-        assert model.run("sparse", m0, m1, None, seed=seed) == "ok"
+        assert model.run("sparse", m0, None, None, seed=seed) == "ok"
     assert failures > 0
+
+
+def test_model_sees_a_missing_merge_handshake():
+    """Block-sparse: without warpgroup 1's wait for merge_free, it can publish the next
+    unit's row maximum and sum over values warpgroup 0 has not read yet."""
+    import importlib.util
+    import os
+    import tempfile
+    src = open(model.__file__).read()
+    a = '''                if u > 0:
+                    yield ("wait", "merge_free", u - 1)
+'''
+    assert src.count(a) == 1
+    d = tempfile.mkdtemp()
+    path = os.path.join(d, "mutant.py")
+    with open(path, "w") as f:
+        f.write(src.replace(a, ""))
+    spec = importlib.util.spec_from_file_location("mutant", path)
+    mutant = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mutant)
+    caught = 0
+    for seed in range(60):
+        try:
+            mutant.run("sparse", [[0], [], [], [1, 2]], None, None, seed=seed)
+        except (mutant.Hazard, mutant.Deadlock):
+            caught += 1
+    assert caught > 0
