@@ -184,8 +184,8 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
  *   block_mask : DEVICE pointer, [ceil(N/128)][ceil(N/128)] bytes, shared by all batches and
  *                heads.
  *   A query that sees no key at all gets O = 0 and lse = -inf.
- *   Runs on the forward kernel of fa_fwd, which streams, for each pair of query tiles, the
- *   union of their active key tiles.
+ *   Runs on the forward kernel of fa_fwd: per query tile, its active key tiles are dealt to
+ *   the kernel's two ping-pong slots in turn and the slots' partial results merged exactly.
  *   workspace : >= fa_fwd_block_sparse_workspace_bytes(B, H, N, d) bytes (the mask packed
  *   into 128 bytes of bits per query tile), 16-byte aligned, caller-owned. */
 size_t fa_fwd_block_sparse_workspace_bytes(int B, int H, int N, int d);
