@@ -131,18 +131,31 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // after it 256-byte aligned.
 constexpr size_t kBwdStatusSlot = 256;
 
-// Split-KV plan: enough (query tile, key slice) units to give every SM of a B200 two (296),
-// at most 64 slices, never more slices than key tiles.  Device-independent, so the
-// workspace size depends on the problem only.
-constexpr long long kSplitTargetUnits = 296;
+// Split-KV plan.  The split kernel runs one CTA per SM (it holds all of TMEM and most of
+// shared memory), and each unit (query tile, key slice) pays a fixed cost (launch, Q load,
+// pipeline fill, partial write) of roughly five key tiles' worth of streaming.  So the plan
+// picks the number of slices n (at most 64, never more than the key tiles) that minimises
+//   rounds(n) * (tiles per slice + 5),  rounds = ceil(units / 148),
+// the time of the busiest SM; ties go to fewer slices (less merging).  Planned for the 148
+// SMs of a B200 whatever the device, so the workspace size depends on the problem only.
+constexpr long long kSplitSlots = 148;
+constexpr long long kSplitUnitCost = 5;  // fixed cost of a unit, in key tiles
 void splitkv_plan(int B, int H, int Nq, int Nk, int* n_split, int* tiles_per_split) {
   const long long kv_tiles = (Nk + 127) / 128;
   const long long base = static_cast<long long>(B) * H * ((Nq + 127) / 128);
-  long long n = (kSplitTargetUnits + base - 1) / base;
-  n = std::max(1LL, std::min(n, std::min(kv_tiles, 64LL)));
-  const long long tps = (kv_tiles + n - 1) / n;
-  *tiles_per_split = static_cast<int>(tps);
-  *n_split = static_cast<int>((kv_tiles + tps - 1) / tps);
+  long long best_cost = -1, best_tps = kv_tiles;
+  for (long long n = 1; n <= std::min(kv_tiles, 64LL); ++n) {
+    const long long tps = (kv_tiles + n - 1) / n;
+    const long long ns = (kv_tiles + tps - 1) / tps;  // slices actually used
+    const long long rounds = (base * ns + kSplitSlots - 1) / kSplitSlots;
+    const long long cost = rounds * (tps + kSplitUnitCost);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_tps = tps;
+    }
+  }
+  *tiles_per_split = static_cast<int>(best_tps);
+  *n_split = static_cast<int>((kv_tiles + best_tps - 1) / best_tps);
 }
 
 int check_splitkv(int B, int H, int Nq, int Nk, int d, int causal, float scale) {

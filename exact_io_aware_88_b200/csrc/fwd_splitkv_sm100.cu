@@ -82,7 +82,8 @@ template <int D, bool CAUSAL, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     splitkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, float* __restrict__ part_o,
-                   float* __restrict__ part_lse, int H, int Nq, int Nk, int n_split,
+                   float* __restrict__ part_lse, void* __restrict__ out, float* __restrict__ lse,
+                   int H, int Nq, int Nk, int n_split,
                    int tiles_per_split, int num_qtiles, int BH, float scale_log2, int* status,
                    uint64_t timeout_ns) {
   using C = Cfg<D>;
@@ -301,7 +302,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- epilogue
     // Partial result of this key slice: O_s = (sum P V) / l and L_s = ln(l) + max (natural
     // log); a row that sees no key of the slice gives O_s = 0, L_s = -inf (weight 0 in the
-    // merge).
+    // merge).  With a single slice the partial result is the result: it goes straight to the
+    // caller's O (bf16 / fp16, [B][Nq][H][D]) and LSE, and no merge runs.
     const size_t prow = (static_cast<size_t>(split) * BH + bh) * Nq + row;
     if (nkv > 0 && ok)
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, 0, ab, status, timeout_ns));
@@ -318,7 +320,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0u;
         }
-        if (row < Nq) {
+        if (row < Nq && n_split == 1) {
+          uint4* dst = reinterpret_cast<uint4*>(
+              static_cast<uint16_t*>(out) + ((static_cast<size_t>(b) * Nq + row) * H + h) * D + 32 * c);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float x0 = __uint_as_float(o[8 * v + 2 * e]) * inv_l;
+              const float x1 = __uint_as_float(o[8 * v + 2 * e + 1]) * inv_l;
+              if constexpr (F16) {
+                const __half2 hv = __floats2half2_rn(x0, x1);
+                w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+              } else {
+                w[e] = pack_bf16x2(x0, x1);
+              }
+            }
+            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else if (row < Nq) {
           float4* dst = reinterpret_cast<float4*>(part_o + prow * D + 32 * c);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
@@ -326,7 +347,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
         }
       }
-      if (row < Nq) part_lse[prow] = have ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      if (row < Nq) {
+        const float L = have ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (n_split == 1)
+          lse[static_cast<size_t>(bh) * Nq + row] = L;
+        else
+          part_lse[prow] = L;
+      }
     }
   }
 
@@ -391,11 +418,12 @@ static cudaError_t launch_t(const SplitKvArgs& a, cudaStream_t st) {
   const long long grid = static_cast<long long>(BH) * num_qtiles * a.n_split;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, st>>>(
-      a.tm_q, a.tm_k, a.tm_v, a.part_o, a.part_lse, a.H, a.Nq, a.Nk, a.n_split,
+      a.tm_q, a.tm_k, a.tm_v, a.part_o, a.part_lse, a.o, a.lse, a.H, a.Nq, a.Nk, a.n_split,
       a.tiles_per_split, num_qtiles, BH, a.scale * 1.4426950408889634f, a.status,
       kDefaultWaitTimeoutNs);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (a.n_split == 1) return cudaSuccess;  // the split kernel wrote O and the LSE itself
   const long long threads = static_cast<long long>(BH) * a.Nq * (D / 4);
   const long long cgrid = (threads + 255) / 256;
   if (F16)
