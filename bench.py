@@ -700,7 +700,8 @@ def run_sweep(path: str, reps: int = 20, warmup: int = 3):
         raise RuntimeError("device status word reports a timeout")
 
 
-KERNEL_CASES = ("fwd_d64_N4096", "fwd_fp8_N4096", "fwd_d128_N4096_causal", "bwd_N4096")
+KERNEL_CASES = ("fwd_d64_N4096", "fwd_fp8_N4096", "fwd_d128_N4096_causal", "bwd_N4096",
+                "bwd_N16384", "decode_k16384", "block_sparse_N16384_d50")
 
 
 def run_kernel_case(name: str, launches: int = 4):
@@ -712,7 +713,11 @@ def run_kernel_case(name: str, launches: int = 4):
       fwd_d128_N4096_causal  the head-dim 128 causal forward (B=4, N=4096, H=16);
       bwd_N4096              one forward, then `launches` backward passes (fa_bwd: its
                              three kernels) on the fwd+bwd workload at N=4096 (B=4, H=16,
-                             d=128, causal).
+                             d=128, causal);
+      bwd_N16384             the same on the bench's workload (B=1, N=16384; ~0.7 GB held);
+      decode_k16384          split-KV decoding, B=8, Nq=1, Nk=16384, H=16, d=128, causal;
+      block_sparse_N16384_d50  the block-sparse forward, B=1, N=16384, H=16, d=128, non-causal,
+                             a random mask of density 0.5 (diagonal kept).
     Prints one line; nothing is timed."""
     import torch
     from exact_io_aware_88_b200 import fa
@@ -722,8 +727,8 @@ def run_kernel_case(name: str, launches: int = 4):
         q, k, v = (t[n].cuda() for n in ("q", "k", "v"))
         for _ in range(launches):
             fa.attention_forward(q, k, v, causal=True)
-    elif name == "bwd_N4096":
-        w = synthetic.fwdbwd(4096)
+    elif name in ("bwd_N4096", "bwd_N16384"):
+        w = synthetic.fwdbwd(4096 if name == "bwd_N4096" else 16384)
         t = synthetic.draw_workload(w, with_grad=True)
         q, k, v, dO = (t[n].cuda() for n in ("q", "k", "v", "dO"))
         o, lse = fa.attention_forward(q, k, v, causal=True)
@@ -733,6 +738,23 @@ def run_kernel_case(name: str, launches: int = 4):
             fa.attention_backward(q, k, v, o, lse, dO, causal=True, workspace=ws)
         if fa.fa_read_device_status(ws) != 0:
             raise RuntimeError("backward status word reports a failure")
+    elif name == "decode_k16384":
+        wl = [x for x in synthetic.decode_workloads() if x[0] == "decode_q1_k16384"][0]
+        _, B, Nq, Nk, H, d, seed = wl
+        t = synthetic.draw_decode(B, Nq, Nk, H, d, seed, "bf16")
+        q, k, v = (t[n].cuda() for n in ("q", "k", "v"))
+        for _ in range(launches):
+            fa.attention_decode(q, k, v, causal=True)
+    elif name == "block_sparse_N16384_d50":
+        B, N, H, d = 1, 16384, 16, 128
+        t = synthetic.draw(B, N, H, d, 1002, "bf16")
+        q, k, v = (t[n].cuda() for n in ("q", "k", "v"))
+        nt = N // 128
+        m = (torch.rand((nt, nt), generator=torch.Generator().manual_seed(77)) < 0.5).to(torch.uint8)
+        m.fill_diagonal_(1)
+        mask = m.cuda()
+        for _ in range(launches):
+            fa.attention_block_sparse(q, k, v, mask, causal=False)
     elif name == "fwd_d64_N4096":
         w = synthetic.fwd_sweep(64, 4096, False)
         t = synthetic.draw_workload(w)
