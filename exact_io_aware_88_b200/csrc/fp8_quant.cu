@@ -7,8 +7,8 @@
 // FlashAttention-3の技術的革新, item 3): rows of Q and K are multiplied by an orthogonal
 // matrix, here M = diag(s) H_d / sqrt(d) with H_d the Sylvester Hadamard matrix, so that
 // (Q M)(K M)^T = Q K^T and rare large entries are spread over all coordinates before the
-// 8-bit rounding.  It is applied as a fast Walsh-Hadamard transform: one warp per row,
-// d/32 elements per lane, log2(d/32) butterfly stages inside a lane and 5 across lanes.
+// 8-bit rounding.  It is applied as a fast Walsh-Hadamard transform: four lanes per row, d/4
+// elements per lane, log2(d/4) butterfly stages inside a lane and 2 across lanes.
 //
 // Two passes, both HBM-bound: (1) the transformed rows' max |x| per (batch, head, tensor)
 // into a workspace (atomicMax on the float bits, valid for non-negative floats); (2) the
@@ -32,29 +32,57 @@ constexpr int kThreads = 256;
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-template <int E>  // elements per lane (d / 32)
-__device__ __forceinline__ void load_row(const __nv_bfloat16* __restrict__ row, int lane,
-                                         float (&x)[E]) {
-  if constexpr (E == 4) {
-    const uint2 u = *reinterpret_cast<const uint2*>(row + lane * 4);
-    x[0] = bf16_lo(u.x);
-    x[1] = bf16_hi(u.x);
-    x[2] = bf16_lo(u.y);
-    x[3] = bf16_hi(u.y);
-  } else {
-    const uint32_t u = *reinterpret_cast<const uint32_t*>(row + lane * 2);
-    x[0] = bf16_lo(u);
-    x[1] = bf16_hi(u);
+// Row layout of passes 1 and 2a: four lanes per row, eight rows per warp (lane = 4 rl + l).
+// Lane l holds the row's 16-byte pieces p = 4c + l (c < D/32), i.e. elements 32c + 8l + k
+// (k < 8), kept at local index e = 8c + k.  The four lanes of a row then load and store
+// contiguous 64-byte runs, and of the transform's log2(d) butterfly stages only the two over
+// index bits 3 and 4 (which lane) need shuffles; the other stages are in-lane adds.
+template <int D>
+struct Quad {
+  static constexpr int E = D / 4;  // elements per lane
+  static constexpr int P = E / 8;  // 16-byte pieces per lane
+};
+
+template <int D>
+__device__ __forceinline__ void load_quad(const __nv_bfloat16* __restrict__ row, int l,
+                                          float (&x)[Quad<D>::E]) {
+#pragma unroll
+  for (int c = 0; c < Quad<D>::P; ++c) {
+    const uint4 u = *reinterpret_cast<const uint4*>(row + 8 * (4 * c + l));
+    x[8 * c + 0] = bf16_lo(u.x);
+    x[8 * c + 1] = bf16_hi(u.x);
+    x[8 * c + 2] = bf16_lo(u.y);
+    x[8 * c + 3] = bf16_hi(u.y);
+    x[8 * c + 4] = bf16_lo(u.z);
+    x[8 * c + 5] = bf16_hi(u.z);
+    x[8 * c + 6] = bf16_lo(u.w);
+    x[8 * c + 7] = bf16_hi(u.w);
   }
 }
 
-// x <- (x * signs) H_d / sqrt(d) for the row spread over the warp (element lane*E + e).
-template <int E>
-__device__ __forceinline__ void hadamard_row(float (&x)[E], const float* __restrict__ signs,
-                                             int lane, float inv_sqrt_d) {
+// Bit e set iff the sign applied to local element e of quarter l is negative.
+template <int D>
+__device__ __forceinline__ uint32_t quad_sign_mask(const float* __restrict__ signs, int l) {
+  uint32_t m = 0u;
 #pragma unroll
-  for (int e = 0; e < E; ++e) x[e] *= signs[lane * E + e];
-  // Index bits inside the lane.
+  for (int c = 0; c < Quad<D>::P; ++c)
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (signs[32 * c + 8 * l + k] < 0.f) m |= 1u << (8 * c + k);
+  return m;
+}
+
+// x <- (x * signs) H_d / sqrt(d) for the row held by the lane's quad.  Local index bits 0-2
+// are global bits 0-2 and local bits 3-4 are global bits 5-6 (in-lane butterflies); global
+// bits 3-4 are the quarter l (shuffles with lanes l ^ 1 and l ^ 2).  The stages commute, so
+// their order does not change the transform.
+template <int D>
+__device__ __forceinline__ void hadamard_quad(float (&x)[Quad<D>::E], uint32_t smask, int lane,
+                                              float inv_sqrt_d) {
+  constexpr int E = Quad<D>::E;
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    x[e] = __uint_as_float(__float_as_uint(x[e]) ^ (((smask >> e) & 1u) << 31));
 #pragma unroll
   for (int h = 1; h < E; h <<= 1) {
 #pragma unroll
@@ -65,9 +93,8 @@ __device__ __forceinline__ void hadamard_row(float (&x)[E], const float* __restr
       x[e + h] = a - b;
     }
   }
-  // Index bits across lanes: the element whose bit is 0 keeps a + b, the other a - b.
 #pragma unroll
-  for (int m = 1; m < 32; m <<= 1) {
+  for (int m = 1; m < 4; m <<= 1) {
     const bool upper = (lane & m) != 0;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -109,9 +136,9 @@ struct Args {
 };
 
 // Work split of passes 1 and 2a: CTA = (tensor, b, h, slice of kRowsPerCta tokens); its 8
-// warps take kUnroll rows at a time so that several row loads are in flight per warp.
+// warps take kUnroll groups of 8 rows at a time so that several loads are in flight per warp.
 constexpr int kRowsPerCta = 512;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 2;  // groups of 8 rows in flight per warp
 
 struct Slice {
   int t, b, h, n0, n1;
@@ -134,23 +161,31 @@ __device__ __forceinline__ const __nv_bfloat16* src_of(const Args& a, int t) {
 // Pass 1: per-head max |x| of the transformed Q, K and of V.
 template <int D>
 __global__ void __launch_bounds__(kThreads) amax_kernel(Args a) {
-  constexpr int E = D / 32;
+  constexpr int E = Quad<D>::E;
   __shared__ float red[kThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rl = lane >> 2, l = lane & 3;
   const Slice s = slice_of(a, blockIdx.x);
   const __nv_bfloat16* base = src_of(a, s.t) + (static_cast<size_t>(s.b) * a.N * a.H + s.h) * D;
   const size_t row_stride = static_cast<size_t>(a.H) * D;
   const bool xf = s.t < 2 && a.signs;
+  const uint32_t smask = xf ? quad_sign_mask<D>(a.signs, l) : 0u;
   float m = 0.f;
-  for (int n = s.n0 + warp * kUnroll; n < s.n1; n += (kThreads / 32) * kUnroll) {
+  for (int n = s.n0 + warp * 8 * kUnroll; n < s.n1; n += (kThreads / 32) * 8 * kUnroll) {
     float x[kUnroll][E];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u)
-      if (n + u < s.n1) load_row<E>(base + (n + u) * row_stride, lane, x[u]);
+    for (int u = 0; u < kUnroll; ++u) {
+      const int row = n + 8 * u + rl;
+      if (row < s.n1) {
+        load_quad<D>(base + row * row_stride, l, x[u]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) x[u][e] = 0.f;
+      }
+    }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      if (n + u >= s.n1) break;
-      if (xf) hadamard_row<E>(x[u], a.signs, lane, a.inv_sqrt_d);
+      if (xf) hadamard_quad<D>(x[u], smask, lane, a.inv_sqrt_d);
 #pragma unroll
       for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(x[u][e]));
     }
@@ -170,33 +205,43 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(Args a) {
 // scales of all three tensors.
 template <int D>
 __global__ void __launch_bounds__(kThreads) quant_qk_kernel(Args a) {
-  constexpr int E = D / 32;
+  constexpr int E = Quad<D>::E;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rl = lane >> 2, l = lane & 3;
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < 3 * a.B * a.H; i += kThreads)
       a.scales[i] = exp2i(scale_exp(__uint_as_float(a.amax[i])));
   const Slice s = slice_of(a, blockIdx.x);
   const size_t head_off = (static_cast<size_t>(s.b) * a.N * a.H + s.h) * D;
   const __nv_bfloat16* base = src_of(a, s.t) + head_off;
-  uint8_t* obase = (s.t == 0 ? a.dst_q : a.dst_k) + head_off + lane * E;
+  uint8_t* obase = (s.t == 0 ? a.dst_q : a.dst_k) + head_off;
   const size_t row_stride = static_cast<size_t>(a.H) * D;
   const float inv = exp2i(-scale_exp(__uint_as_float(a.amax[s.t * a.B * a.H + s.b * a.H + s.h])));
-  for (int n = s.n0 + warp * kUnroll; n < s.n1; n += (kThreads / 32) * kUnroll) {
+  const uint32_t smask = a.signs ? quad_sign_mask<D>(a.signs, l) : 0u;
+  for (int n = s.n0 + warp * 8 * kUnroll; n < s.n1; n += (kThreads / 32) * 8 * kUnroll) {
     float x[kUnroll][E];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u)
-      if (n + u < s.n1) load_row<E>(base + (n + u) * row_stride, lane, x[u]);
+    for (int u = 0; u < kUnroll; ++u) {
+      const int row = n + 8 * u + rl;
+      if (row < s.n1) {
+        load_quad<D>(base + row * row_stride, l, x[u]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) x[u][e] = 0.f;
+      }
+    }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      if (n + u >= s.n1) break;
-      if (a.signs) hadamard_row<E>(x[u], a.signs, lane, a.inv_sqrt_d);
-      uint8_t* out = obase + (n + u) * row_stride;
-      if constexpr (E == 4) {
-        const uint32_t lo = pack_e4m3x2(x[u][0] * inv, x[u][1] * inv);
-        const uint32_t hi = pack_e4m3x2(x[u][2] * inv, x[u][3] * inv);
-        *reinterpret_cast<uint32_t*>(out) = lo | (hi << 16);
-      } else {
-        *reinterpret_cast<uint16_t*>(out) = static_cast<uint16_t>(pack_e4m3x2(x[u][0] * inv, x[u][1] * inv));
+      if (a.signs) hadamard_quad<D>(x[u], smask, lane, a.inv_sqrt_d);
+      const int row = n + 8 * u + rl;
+      if (row >= s.n1) continue;
+      uint8_t* out = obase + row * row_stride;
+#pragma unroll
+      for (int c = 0; c < Quad<D>::P; ++c) {
+        const float* v = &x[u][8 * c];
+        const uint32_t w0 = pack_e4m3x2(v[0] * inv, v[1] * inv) | (pack_e4m3x2(v[2] * inv, v[3] * inv) << 16);
+        const uint32_t w1 = pack_e4m3x2(v[4] * inv, v[5] * inv) | (pack_e4m3x2(v[6] * inv, v[7] * inv) << 16);
+        *reinterpret_cast<uint2*>(out + 8 * (4 * c + l)) = make_uint2(w0, w1);
       }
     }
   }
