@@ -17,8 +17,16 @@
 // and writes dQ_i = scale * dQ_i in bf16.  Cost: the S and dP products are computed a second
 // time (the main kernel computes them too), 1.4x the tensor work of the atomic variant.
 //
+// S has two TMEM buffers, used by key tiles in turn, so the S product of tile j+2 is issued
+// as soon as dQ of tile j (which reads dS_j from the same columns) is: per key tile, in issue
+// order, [ds_ready j] dP(j+1), dQ(j), S(j+2).  The compute warps then wait on one product
+// (dP) between tiles instead of three, and the tensor core runs S ahead of them.  K is read
+// by S(j) and, two issue steps later, dQ(j), so it has a three-stage ring; V, read by dP(j)
+// only, two stages.
+//
 // CTA = 6 warps: 0-3 compute (thread t owns query row t = TMEM lane t), 4 TMA producer,
-// 5 TMEM allocator + MMA issuer.  TMEM: S / dS [0,128), dP [128,256), dQ [256,256+D).
+// 5 TMEM allocator + MMA issuer.  TMEM: S / dS buffer 0 [0,128), dP [128,256),
+// dQ [256,256+D), S / dS buffer 1 [384,512).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -34,26 +42,31 @@ constexpr int BM = 128;  // query rows per CTA
 constexpr int BN = 128;  // key rows per step
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
+constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColS1 = 384;
+// TMEM column of S / dS buffer b (key tile j uses buffer j % 2).
+__host__ __device__ constexpr uint32_t col_s(int b) { return b ? kColS1 : kColS; }
 
 template <int D>
 struct Cfg {
   static constexpr int kChunks = D / 64;
   static constexpr int kChunkBytes = 128 * 128;  // one TMA box: 128 rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStages = 2;              // K/V ring
+  static constexpr int kKStages = 3;             // K ring (read two issue steps apart)
+  static constexpr int kVStages = 2;             // V ring
   static constexpr int kOffQ = 0;
   static constexpr int kOffDO = kOffQ + kTileBytes;
   static constexpr int kOffK = kOffDO + kTileBytes;
-  static constexpr int kOffV = kOffK + kStages * kTileBytes;
-  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
   static constexpr int kSmemBytes = kOffBar + 256;  // base is 1024-aligned (checked)
+  static_assert(kSmemBytes <= 232448, "more shared memory than a CTA can have");
 };
 
 struct Bars {
   uint64_t qd_full;
-  uint64_t k_full[2], v_full[2], kv_empty[2];
-  uint64_t s_full, dp_full, ds_ready, dq_done, drain;
+  uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
+  uint64_t s_full[2];  // per S buffer: one phase per use, so it never runs ahead of its waiter
+  uint64_t dp_full, ds_ready, dq_done, drain;
   uint32_t tmem_base;
   Abort abort;
 };
@@ -87,12 +100,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->qd_full, 1);
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < C::kKStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
     }
-    mbar_init(&bars->s_full, 1);
+    for (int s = 0; s < C::kVStages; ++s) {
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    mbar_init(&bars->s_full[0], 1);
+    mbar_init(&bars->s_full[1], 1);
     mbar_init(&bars->dp_full, 1);
     mbar_init(&bars->ds_ready, BM);
     mbar_init(&bars->dq_done, 1);
@@ -128,53 +145,63 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(sQ + c * C::kChunkBytes, &tm_q, &bars->qd_full, c * 64, h, q0, b, pol_q);
         tma_load_4d(sDO + c * C::kChunkBytes, &tm_do, &bars->qd_full, c * 64, h, q0, b, pol_q);
       }
-      int issued = 0;
+      int k_issued = 0, v_issued = 0;
       for (int j = 0; j < nkv; ++j) {
-        const int s = j % C::kStages;
-        if (j >= C::kStages &&
-            !mbar_wait(&bars->kv_empty[s], ((j / C::kStages) - 1) & 1, ab, status, timeout_ns))
+        const int sk = j % C::kKStages, sv = j % C::kVStages;
+        if (j >= C::kKStages &&
+            !mbar_wait(&bars->k_empty[sk], ((j / C::kKStages) - 1) & 1, ab, status, timeout_ns))
           break;
-        mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes);
+        mbar_arrive_expect_tx(&bars->k_full[sk], C::kTileBytes);
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sK + s * C::kTileBytes + c * C::kChunkBytes, &tm_k, &bars->k_full[s], c * 64,
+          tma_load_4d(sK + sk * C::kTileBytes + c * C::kChunkBytes, &tm_k, &bars->k_full[sk], c * 64,
                       h, j * BN, b, pol_kv);
-        mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
+        k_issued = j + 1;
+        if (j >= C::kVStages &&
+            !mbar_wait(&bars->v_empty[sv], ((j / C::kVStages) - 1) & 1, ab, status, timeout_ns))
+          break;
+        mbar_arrive_expect_tx(&bars->v_full[sv], C::kTileBytes);
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sV + s * C::kTileBytes + c * C::kChunkBytes, &tm_v, &bars->v_full[s], c * 64,
+          tma_load_4d(sV + sv * C::kTileBytes + c * C::kChunkBytes, &tm_v, &bars->v_full[sv], c * 64,
                       h, j * BN, b, pol_kv);
-        issued = j + 1;
+        v_issued = j + 1;
       }
+      // Drain every copy into shared memory before the CTA may exit.
       Abort local{0};
       mbar_wait(&bars->qd_full, 0, &local, status, timeout_ns);
-      for (int j = max(0, issued - C::kStages); j < issued; ++j) {
-        mbar_wait(&bars->k_full[j % C::kStages], (j / C::kStages) & 1, &local, status, timeout_ns);
-        mbar_wait(&bars->v_full[j % C::kStages], (j / C::kStages) & 1, &local, status, timeout_ns);
-      }
+      for (int j = max(0, k_issued - C::kKStages); j < k_issued; ++j)
+        mbar_wait(&bars->k_full[j % C::kKStages], (j / C::kKStages) & 1, &local, status, timeout_ns);
+      for (int j = max(0, v_issued - C::kVStages); j < v_issued; ++j)
+        mbar_wait(&bars->v_full[j % C::kVStages], (j / C::kVStages) & 1, &local, status, timeout_ns);
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------------ MMA issuer
-    // Per key tile j: S, dP; [ds_ready j] dQ += dS K_j.  S(j+1) overwrites the dS columns
-    // only after dQ(j) has read them (tcgen05 operations of one thread run in order).
+    // Prologue S(0), dP(0), S(1); then per key tile j: [ds_ready j] dP(j+1), dQ(j) += dS_j K_j,
+    // S(j+2).  S(j+2) overwrites buffer j % 2 after dQ(j) has read dS_j from it, and dP(j+1)
+    // overwrites dP_j after the compute warps have read it (ds_ready j): tcgen05 operations of
+    // one thread run in order.
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16_f32(BM, BN, 0, 0);   // Q K^T, dO V^T (K-major)
       constexpr uint32_t id_dq = idesc_bf16_f32(BM, D, 0, 1);   // dS K (B MN-major)
       const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV);
-      bool ok = mbar_wait(&bars->qd_full, 0, ab, status, timeout_ns);
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j % C::kStages;
-        const uint32_t ph = (j / C::kStages) & 1;
-        if (!(ok = mbar_wait(&bars->k_full[s], ph, ab, status, timeout_ns))) break;
+      auto issue_s = [&](int j) -> bool {
+        const int sk = j % C::kKStages;
+        if (!mbar_wait(&bars->k_full[sk], (j / C::kKStages) & 1, ab, status, timeout_ns)) return false;
         tc_fence_after();
-        const uint32_t kb = aK + s * C::kTileBytes, vb = aV + s * C::kTileBytes;
+        const uint32_t kb = aK + sk * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-          umma_ss(tbase + kColS, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
-                  id_s, kk > 0);
+          umma_ss(tbase + col_s(j & 1), sdesc_sw128(aQ + off, 16, 1024),
+                  sdesc_sw128(kb + off, 16, 1024), id_s, kk > 0);
         }
-        umma_commit(&bars->s_full);
-        if (!(ok = mbar_wait(&bars->v_full[s], ph, ab, status, timeout_ns))) break;
+        umma_commit(&bars->s_full[j & 1]);
+        return true;
+      };
+      auto issue_dp = [&](int j) -> bool {
+        const int sv = j % C::kVStages;
+        if (!mbar_wait(&bars->v_full[sv], (j / C::kVStages) & 1, ab, status, timeout_ns)) return false;
         tc_fence_after();
+        const uint32_t vb = aV + sv * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
@@ -182,13 +209,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                   id_s, kk > 0);
         }
         umma_commit(&bars->dp_full);
+        umma_commit(&bars->v_empty[sv]);  // dP is V's only reader
+        return true;
+      };
+      bool ok = mbar_wait(&bars->qd_full, 0, ab, status, timeout_ns) && issue_s(0) && issue_dp(0) &&
+                (nkv < 2 || issue_s(1));
+      for (int j = 0; ok && j < nkv; ++j) {
         if (!(ok = mbar_wait(&bars->ds_ready, j & 1, ab, status, timeout_ns))) break;
         tc_fence_after();
+        if (j + 1 < nkv && !(ok = issue_dp(j + 1))) break;
+        const int sk = j % C::kKStages;
+        const uint32_t kb = aK + sk * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts(tbase + kColDQ, tbase + kColS + kk * 8,
+          umma_ts(tbase + kColDQ, tbase + col_s(j & 1) + kk * 8,
                   sdesc_sw128(kb + kk * 2048, C::kChunkBytes, 1024), id_dq, (j > 0 || kk > 0));
-        umma_commit(&bars->kv_empty[s]);
+        umma_commit(&bars->k_empty[sk]);  // dQ(j) is K_j's last reader
+        if (j + 2 < nkv && !(ok = issue_s(j + 2))) break;
       }
       umma_commit(&bars->dq_done);
       umma_commit(&bars->drain);
@@ -205,19 +242,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float dd = delta[vec];
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, ab, status, timeout_ns));
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, ab, status, timeout_ns));
       if (!ok) break;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, j & 1, ab, status, timeout_ns));
       if (!ok) break;
       tc_fence_after();
       const int k0 = j * BN;
+      const uint32_t colS = col_s(j & 1);
       const int lim = min(CAUSAL ? row : N - 1, N - 1) - k0;  // last visible key column
       const bool need_mask = lim < BN - 1;
       const bool masked = __any_sync(0xffffffffu, need_mask);
 #pragma unroll
       for (int c32 = 0; c32 < BN / 32; ++c32) {
         uint32_t su[32], du[32];
-        tmem_ld32(lane_base + kColS + 32 * c32, su);
+        tmem_ld32(lane_base + colS + 32 * c32, su);
         tmem_ld32(lane_base + kColDP + 32 * c32, du);
         uint32_t pk[16];
 #pragma unroll
@@ -231,9 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[e / 2] = pack_bf16x2(p0 * (__uint_as_float(du[e]) - dd),
                                   p1 * (__uint_as_float(du[e + 1]) - dd));
         }
-        // dS (bf16 pairs) into columns [16 c32, 16 c32 + 16) of the S region: inside the S
-        // columns already read (this chunk or an earlier one).
-        tmem_st16(lane_base + kColS + 16 * c32, pk);
+        // dS (bf16 pairs) into columns [16 c32, 16 c32 + 16) of this tile's S buffer: inside
+        // the S columns already read (this chunk or an earlier one).
+        tmem_st16(lane_base + colS + 16 * c32, pk);
       }
       tmem_st_wait();
       tc_fence_before();
