@@ -44,11 +44,11 @@ constexpr int BN = 128;  // query rows per step
 constexpr int kThreads = 512;
 // 16 warps = 4 warpgroups; sub-partition k runs warps k, k+4, k+8, k+12, one from each
 // warpgroup.  Launch gives 128 registers to every thread (65536); after setmaxnreg each
-// sub-partition holds 152 + 152 + 136 + 72 = 512 registers per lane (= 512 launched).
+// sub-partition holds 144 + 144 + 136 + 88 = 512 registers per lane (= 512 launched).
 constexpr uint32_t kRegsLaunch = 65536 / kThreads;  // 128 (ptxas allocates this at launch)
-constexpr uint32_t kRegsCompute = 152;
+constexpr uint32_t kRegsCompute = 144;
 constexpr uint32_t kRegsDrain = 136;
-constexpr uint32_t kRegsOther = 72;
+constexpr uint32_t kRegsOther = 88;
 static_assert(2 * kRegsCompute + kRegsDrain + kRegsOther <= 4 * kRegsLaunch,
               "register split exceeds what the block is launched with");
 constexpr int kWarpLoad = 12;
@@ -435,19 +435,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t id_dq = kDqTransposed<D>
                                        ? idesc_bf16_f32(D, BN, 1, 1)   // K_j^T dS^T
                                        : idesc_bf16_f32(BN, D, 1, 1);  // dS K_j
-        const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ),
-                       aDO = smem_u32(sDO), aDS = smem_u32(sDS);
+        // Low descriptor words of the operand tiles read K-major (rows of the head dim, or of
+        // the query index for dS^T: LBO unused); the Q and dO stages are offsets from the
+        // first.  kdesc(x, off) / mdesc(x, off) describe the operand `off` bytes into tile x
+        // read K-major / MN-major (LBO = one 64-column chunk).
+        constexpr uint32_t kHi = sdesc_sw128_hi(1024);
+        constexpr uint32_t kToMn = ((C::kChunkBytes >> 4) - 1u) << 16;  // LBO 16 -> chunk
+        const uint32_t xK = sdesc_sw128_lo(smem_u32(sK), 16);
+        const uint32_t xV = sdesc_sw128_lo(smem_u32(sV), 16);
+        const uint32_t xQ0 = sdesc_sw128_lo(smem_u32(sQ), 16);
+        const uint32_t xDO0 = sdesc_sw128_lo(smem_u32(sDO), 16);
+        const uint32_t xDS = sdesc_sw128_lo(smem_u32(sDS), 16);
+        auto kdesc = [](uint32_t x, uint32_t off) { return sdesc_join(x + (off >> 4), kHi); };
+        auto mdesc = [](uint32_t x, uint32_t off) { return sdesc_join(x + (off >> 4) + kToMn, kHi); };
         auto issue_s = [&](int n) -> bool {  // S^T_n = K_j Q_n^T (K-major over the head dim)
           const int sq = n % C::kQStages;
           if (!mbar_wait(&bars->q_full[sq], (n / C::kQStages) & 1, ab, status, timeout_ns))
             return false;
           tc_fence_after();
-          const uint32_t qb = aQ + sq * C::kTileBytes;
+          const uint32_t qd = xQ0 + ((sq * C::kTileBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-            umma_ss(tbase + C::kColS, sdesc_sw128(aK + off, 16, 1024),
-                    sdesc_sw128(qb + off, 16, 1024), id_sdp, kk > 0);
+            umma_ss(tbase + C::kColS, kdesc(xK, off), kdesc(qd, off), id_sdp, kk > 0);
           }
           umma_commit(&bars->s_full);
           return true;
@@ -459,12 +469,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (WITH_DQ && n > 0 && !mbar_wait(&bars->dq_empty, (n - 1) & 1, ab, status, timeout_ns))
             return false;
           tc_fence_after();
-          const uint32_t dob = aDO + sd * C::kTileBytes;
+          const uint32_t dod = xDO0 + ((sd * C::kTileBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-            umma_ss(tbase + C::kColDP, sdesc_sw128(aV + off, 16, 1024),
-                    sdesc_sw128(dob + off, 16, 1024), id_sdp, kk > 0);
+            umma_ss(tbase + C::kColDP, kdesc(xV, off), kdesc(dod, off), id_sdp, kk > 0);
           }
           umma_commit(&bars->dp_full);
           return true;
@@ -473,14 +482,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         int mma_steps = 0;
         for (int n = 0; ok && n < nq; ++n) {
           const int sq = n % C::kQStages, sd = n % C::kDOStages;
-          const uint32_t qb = aQ + sq * C::kTileBytes, dob = aDO + sd * C::kTileBytes;
+          const uint32_t xq = xQ0 + ((sq * C::kTileBytes) >> 4);
+          const uint32_t xdo = xDO0 + ((sd * C::kTileBytes) >> 4);
           if (!mbar_wait(&bars->p_ready, n & 1, ab, status, timeout_ns)) break;
           tc_fence_after();
           // dV_j += P^T dO_i   (A = P^T from TMEM, B = dO_i MN-major over the query index)
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
             umma_ts(tbase + C::kColDV, tbase + C::kColS + p_col(kk),
-                    sdesc_sw128(dob + kk * 2048, C::kChunkBytes, 1024), id_dkdv, (n > 0 || kk > 0));
+                    mdesc(xdo, kk * 2048), id_dkdv, (n > 0 || kk > 0));
           umma_commit(&bars->do_empty[sd]);
           if (n + 1 < nq && !issue_s(n + 1)) break;
           if (!mbar_wait(&bars->ds_ready, n & 1, ab, status, timeout_ns)) break;
@@ -493,22 +503,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             // MN-major over the query index): TMEM lane = head-dim index, column = query.
 #pragma unroll
             for (int kk = 0; kk < BM / 16; ++kk)
-              umma_ss(tbase + C::kColDP, sdesc_sw128(aK + kk * 2048, C::kChunkBytes, 1024),
-                      sdesc_sw128(aDS + kk * 2048, C::kChunkBytes, 1024), id_dq, kk > 0);
+              umma_ss(tbase + C::kColDP, mdesc(xK, kk * 2048), mdesc(xDS, kk * 2048), id_dq, kk > 0);
           } else {
             // dQ_i = dS K_j   (A = dS: the dS^T tile read MN-major; B = K_j MN-major)
 #pragma unroll
             for (int kk = 0; kk < BM / 16; ++kk)
-              umma_ss(tbase + C::kColDP, sdesc_sw128(aDS + kk * 2048, C::kChunkBytes, 1024),
-                      sdesc_sw128(aK + kk * 2048, C::kChunkBytes, 1024), id_dq, kk > 0);
+              umma_ss(tbase + C::kColDP, mdesc(xDS, kk * 2048), mdesc(xK, kk * 2048), id_dq, kk > 0);
           }
           if constexpr (WITH_DQ) umma_commit(&bars->dq_full);
           // dK_j += dS^T Q_i   (A = dS^T K-major over the query index, B = Q_i MN-major)
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
             const uint32_t aoff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-            umma_ss(tbase + C::kColDK, sdesc_sw128(aDS + aoff, 16, 1024),
-                    sdesc_sw128(qb + kk * 2048, C::kChunkBytes, 1024), id_dkdv, (n > 0 || kk > 0));
+            umma_ss(tbase + C::kColDK, kdesc(xDS, aoff), mdesc(xq, kk * 2048), id_dkdv,
+                    (n > 0 || kk > 0));
           }
           umma_commit(&bars->q_empty[sq]);
           ++mma_steps;

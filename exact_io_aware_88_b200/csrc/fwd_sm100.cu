@@ -737,7 +737,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t idesc_s = F8 ? idesc_e4m3_f32(BM, BN, 0, 0) : idesc_bf16_f32(BM, BN, 0, 0);
         // PV: bf16 V is [keys][d] (MN-major B); the 8-bit V^T is [d][keys] (K-major B).
         constexpr uint32_t idesc_o = F8 ? idesc_e4m3_f32(BM, D, 0, 0) : idesc_bf16_f32(BM, D, 0, 1);
-        const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+        // Descriptors of the first Q, K and V tiles; the others are offsets from them.
+        const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+        const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+        const uint64_t dV0 = sdesc_sw128(smem_u32(sV), F8 ? 16 : C::kChunkBytes, 1024);
         int g = 0;            // K/V tiles consumed so far (ring position)
         int units = 0;        // units finished
         int np[2] = {0, 0};   // p_full phases consumed per tile
@@ -745,37 +748,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         int s_issued0 = 0, s_issued1 = 0;  // S products issued per tile (protocol check)
         auto issue_s = [&](int t, int s) {  // S_t = Q_t K^T (both K-major over the head dim)
           (t ? s_issued1 : s_issued0) += 1;
-          const uint32_t kb = aK + s * C::kTileBytes;
-          const uint32_t qb = aQ + (SPARSE ? 0 : t * C::kTileBytes);  // sparse: one Q, both slots
+          const uint64_t kd = sdesc_advance(dK0, s * C::kTileBytes);
+          const uint64_t qd = sdesc_advance(dQ0, SPARSE ? 0 : t * C::kTileBytes);  // sparse: one Q
           // One MMA per 32 bytes of the head dim (16 bf16 or 32 E4M3 elements).
 #pragma unroll
           for (int kk = 0; kk < C::kRowBytes / 32; ++kk) {
             const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
             if constexpr (F8)
-              umma_ss_f8(tbase + BN * t, sdesc_sw128(qb + off, 16, 1024),
-                         sdesc_sw128(kb + off, 16, 1024), idesc_s, kk > 0);
+              umma_ss_f8(tbase + BN * t, sdesc_advance(qd, off), sdesc_advance(kd, off), idesc_s,
+                         kk > 0);
             else
-              umma_ss(tbase + BN * t, sdesc_sw128(qb + off, 16, 1024),
-                      sdesc_sw128(kb + off, 16, 1024), idesc_s, kk > 0);
+              umma_ss(tbase + BN * t, sdesc_advance(qd, off), sdesc_advance(kd, off), idesc_s,
+                      kk > 0);
           }
           umma_commit(&bars->s_full[t]);
         };
         // O_t += P_t V over keys [64 h, 64 h + 64) of the tile (P from TMEM).
         auto issue_pv_half = [&](int t, int s, bool first, int h) {
-          const uint32_t vb = aV + s * C::kTileBytes;
+          const uint64_t vd = sdesc_advance(dV0, s * C::kTileBytes);
           if constexpr (F8) {  // 32 keys per MMA: 8 TMEM columns of P, 32 bytes of V^T rows
 #pragma unroll
             for (int k2 = 0; k2 < BN / 64; ++k2) {
               const int kk = h * (BN / 64) + k2;
               umma_ts_f8(tbase + C::kColO + 128 * t, tbase + BN * t + kk * 8,
-                         sdesc_sw128(vb + kk * 32, 16, 1024), idesc_o, (!first || kk > 0) ? 1u : 0u);
+                         sdesc_advance(vd, kk * 32), idesc_o, (!first || kk > 0) ? 1u : 0u);
             }
           } else {
 #pragma unroll
             for (int k2 = 0; k2 < BN / 32; ++k2) {
               const int kk = h * (BN / 32) + k2;
               umma_ts(tbase + C::kColO + 128 * t, tbase + BN * t + kk * 8,
-                      sdesc_sw128(vb + kk * 2048, C::kChunkBytes, 1024), idesc_o,
+                      sdesc_advance(vd, kk * 2048), idesc_o,
                       (!first || kk > 0) ? 1u : 0u);
             }
           }

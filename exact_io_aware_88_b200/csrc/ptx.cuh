@@ -284,6 +284,28 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// The descriptor of the operand `byte_off` bytes past the one `d` describes, in the same
+// layout: only the start address (bits [0,14), in 16-byte units) moves, and shared-memory
+// addresses (below 256 KB) never carry out of that field.  One add instead of rebuilding the
+// descriptor, for the MMA-issuing thread whose instruction latency is on the critical path.
+__device__ __forceinline__ uint64_t sdesc_advance(uint64_t d, uint32_t byte_off) {
+  return d + (byte_off >> 4);
+}
+
+// sdesc_sw128's descriptor as two 32-bit words, for a thread short of registers: the low word
+// (start address and LBO) per operand, the high word (SBO, version, layout) a constant.
+// sdesc_join(sdesc_sw128_lo(a, lbo) + (off >> 4), sdesc_sw128_hi(sbo)) equals
+// sdesc_sw128(a + off, lbo, sbo) for shared-memory addresses, as in sdesc_advance.
+__device__ __forceinline__ uint32_t sdesc_sw128_lo(uint32_t saddr, uint32_t lbo) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t sdesc_sw128_hi(uint32_t sbo) {
+  return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+__device__ __forceinline__ uint64_t sdesc_join(uint32_t lo, uint32_t hi) {
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D, dense.
 //   [4,6) D format = 1 (f32)   [7,10) A format = 1 (bf16)   [10,13) B format = 1 (bf16)
 //   [15] A major (0 K, 1 MN)   [16] B major   [17,23) N >> 3   [24,29) M >> 4
