@@ -182,17 +182,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16_f32(BM, BN, 0, 0);   // Q K^T, dO V^T (K-major)
       constexpr uint32_t id_dq = idesc_bf16_f32(BM, D, 0, 1);   // dS K (B MN-major)
-      const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV);
+      // Low descriptor words of the operand tiles read K-major; the K and V stages are offsets
+      // from the first.  kdesc / mdesc: K-major / MN-major (LBO = one 64-column chunk).
+      constexpr uint32_t kHi = sdesc_sw128_hi(1024);
+      constexpr uint32_t kToMn = ((C::kChunkBytes >> 4) - 1u) << 16;
+      const uint32_t xQ = sdesc_sw128_lo(smem_u32(sQ), 16), xDO = sdesc_sw128_lo(smem_u32(sDO), 16);
+      const uint32_t xK0 = sdesc_sw128_lo(smem_u32(sK), 16), xV0 = sdesc_sw128_lo(smem_u32(sV), 16);
+      auto kdesc = [](uint32_t x, uint32_t off) { return sdesc_join(x + (off >> 4), kHi); };
+      auto mdesc = [](uint32_t x, uint32_t off) { return sdesc_join(x + (off >> 4) + kToMn, kHi); };
       auto issue_s = [&](int j) -> bool {
         const int sk = j % C::kKStages;
         if (!mbar_wait(&bars->k_full[sk], (j / C::kKStages) & 1, ab, status, timeout_ns)) return false;
         tc_fence_after();
-        const uint32_t kb = aK + sk * C::kTileBytes;
+        const uint32_t xk = xK0 + ((sk * C::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-          umma_ss(tbase + col_s(j & 1), sdesc_sw128(aQ + off, 16, 1024),
-                  sdesc_sw128(kb + off, 16, 1024), id_s, kk > 0);
+          umma_ss(tbase + col_s(j & 1), kdesc(xQ, off), kdesc(xk, off), id_s, kk > 0);
         }
         umma_commit(&bars->s_full[j & 1]);
         return true;
@@ -201,12 +207,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sv = j % C::kVStages;
         if (!mbar_wait(&bars->v_full[sv], (j / C::kVStages) & 1, ab, status, timeout_ns)) return false;
         tc_fence_after();
-        const uint32_t vb = aV + sv * C::kTileBytes;
+        const uint32_t xv = xV0 + ((sv * C::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-          umma_ss(tbase + kColDP, sdesc_sw128(aDO + off, 16, 1024), sdesc_sw128(vb + off, 16, 1024),
-                  id_s, kk > 0);
+          umma_ss(tbase + kColDP, kdesc(xDO, off), kdesc(xv, off), id_s, kk > 0);
         }
         umma_commit(&bars->dp_full);
         umma_commit(&bars->v_empty[sv]);  // dP is V's only reader
@@ -219,11 +224,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (j + 1 < nkv && !(ok = issue_dp(j + 1))) break;
         const int sk = j % C::kKStages;
-        const uint32_t kb = aK + sk * C::kTileBytes;
+        const uint32_t xk = xK0 + ((sk * C::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts(tbase + kColDQ, tbase + col_s(j & 1) + kk * 8,
-                  sdesc_sw128(kb + kk * 2048, C::kChunkBytes, 1024), id_dq, (j > 0 || kk > 0));
+          umma_ts(tbase + kColDQ, tbase + col_s(j & 1) + kk * 8, mdesc(xk, kk * 2048), id_dq,
+                  (j > 0 || kk > 0));
         umma_commit(&bars->k_empty[sk]);  // dQ(j) is K_j's last reader
         if (j + 2 < nkv && !(ok = issue_s(j + 2))) break;
       }
