@@ -43,20 +43,26 @@ struct Quad {
   static constexpr int P = E / 8;  // 16-byte pieces per lane
 };
 
+// The lane's pieces of one row as raw bf16 words (loads only), and their widening to fp32.
+// Split so that a warp can have the next rows' loads in flight while it transforms these.
 template <int D>
-__device__ __forceinline__ void load_quad(const __nv_bfloat16* __restrict__ row, int l,
-                                          float (&x)[Quad<D>::E]) {
+__device__ __forceinline__ void fetch_quad(const __nv_bfloat16* __restrict__ row, int l,
+                                           uint4 (&r)[Quad<D>::P]) {
+#pragma unroll
+  for (int c = 0; c < Quad<D>::P; ++c) r[c] = *reinterpret_cast<const uint4*>(row + 8 * (4 * c + l));
+}
+template <int D>
+__device__ __forceinline__ void widen_quad(const uint4 (&r)[Quad<D>::P], float (&x)[Quad<D>::E]) {
 #pragma unroll
   for (int c = 0; c < Quad<D>::P; ++c) {
-    const uint4 u = *reinterpret_cast<const uint4*>(row + 8 * (4 * c + l));
-    x[8 * c + 0] = bf16_lo(u.x);
-    x[8 * c + 1] = bf16_hi(u.x);
-    x[8 * c + 2] = bf16_lo(u.y);
-    x[8 * c + 3] = bf16_hi(u.y);
-    x[8 * c + 4] = bf16_lo(u.z);
-    x[8 * c + 5] = bf16_hi(u.z);
-    x[8 * c + 6] = bf16_lo(u.w);
-    x[8 * c + 7] = bf16_hi(u.w);
+    x[8 * c + 0] = bf16_lo(r[c].x);
+    x[8 * c + 1] = bf16_hi(r[c].x);
+    x[8 * c + 2] = bf16_lo(r[c].y);
+    x[8 * c + 3] = bf16_hi(r[c].y);
+    x[8 * c + 4] = bf16_lo(r[c].z);
+    x[8 * c + 5] = bf16_hi(r[c].z);
+    x[8 * c + 6] = bf16_lo(r[c].w);
+    x[8 * c + 7] = bf16_hi(r[c].w);
   }
 }
 
@@ -136,9 +142,29 @@ struct Args {
 };
 
 // Work split of passes 1 and 2a: CTA = (tensor, b, h, slice of kRowsPerCta tokens); its 8
-// warps take kUnroll groups of 8 rows at a time so that several loads are in flight per warp.
+// warps take kUnroll groups of 8 rows at a time, and the loads of a warp's next groups are
+// issued before it transforms the current ones, so that DRAM reads never stop while the
+// warp computes.
 constexpr int kRowsPerCta = 512;
-constexpr int kUnroll = 2;  // groups of 8 rows in flight per warp
+constexpr int kUnroll = 1;  // groups of 8 rows per step of a warp (two: 171 registers at d=128)
+constexpr int kRowStep = (kThreads / 32) * 8 * kUnroll;  // rows a CTA takes per step
+
+// The raw words of a warp's kUnroll groups starting at row n (rows past n1 read as zeros).
+template <int D>
+__device__ __forceinline__ void fetch_groups(const __nv_bfloat16* __restrict__ base,
+                                             size_t row_stride, int n, int n1, int rl, int l,
+                                             uint4 (&r)[kUnroll][Quad<D>::P]) {
+#pragma unroll
+  for (int u = 0; u < kUnroll; ++u) {
+    const int row = n + 8 * u + rl;
+    if (row < n1) {
+      fetch_quad<D>(base + row * row_stride, l, r[u]);
+    } else {
+#pragma unroll
+      for (int c = 0; c < Quad<D>::P; ++c) r[u][c] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+}
 
 struct Slice {
   int t, b, h, n0, n1;
@@ -171,18 +197,14 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(Args a) {
   const bool xf = s.t < 2 && a.signs;
   const uint32_t smask = xf ? quad_sign_mask<D>(a.signs, l) : 0u;
   float m = 0.f;
-  for (int n = s.n0 + warp * 8 * kUnroll; n < s.n1; n += (kThreads / 32) * 8 * kUnroll) {
+  uint4 raw[kUnroll][Quad<D>::P];
+  int n = s.n0 + warp * 8 * kUnroll;
+  if (n < s.n1) fetch_groups<D>(base, row_stride, n, s.n1, rl, l, raw);
+  for (; n < s.n1; n += kRowStep) {
     float x[kUnroll][E];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int row = n + 8 * u + rl;
-      if (row < s.n1) {
-        load_quad<D>(base + row * row_stride, l, x[u]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < E; ++e) x[u][e] = 0.f;
-      }
-    }
+    for (int u = 0; u < kUnroll; ++u) widen_quad<D>(raw[u], x[u]);
+    if (n + kRowStep < s.n1) fetch_groups<D>(base, row_stride, n + kRowStep, s.n1, rl, l, raw);
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       if (xf) hadamard_quad<D>(x[u], smask, lane, a.inv_sqrt_d);
@@ -218,18 +240,14 @@ __global__ void __launch_bounds__(kThreads) quant_qk_kernel(Args a) {
   const size_t row_stride = static_cast<size_t>(a.H) * D;
   const float inv = exp2i(-scale_exp(__uint_as_float(a.amax[s.t * a.B * a.H + s.b * a.H + s.h])));
   const uint32_t smask = a.signs ? quad_sign_mask<D>(a.signs, l) : 0u;
-  for (int n = s.n0 + warp * 8 * kUnroll; n < s.n1; n += (kThreads / 32) * 8 * kUnroll) {
+  uint4 raw[kUnroll][Quad<D>::P];
+  int n = s.n0 + warp * 8 * kUnroll;
+  if (n < s.n1) fetch_groups<D>(base, row_stride, n, s.n1, rl, l, raw);
+  for (; n < s.n1; n += kRowStep) {
     float x[kUnroll][E];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int row = n + 8 * u + rl;
-      if (row < s.n1) {
-        load_quad<D>(base + row * row_stride, l, x[u]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < E; ++e) x[u][e] = 0.f;
-      }
-    }
+    for (int u = 0; u < kUnroll; ++u) widen_quad<D>(raw[u], x[u]);
+    if (n + kRowStep < s.n1) fetch_groups<D>(base, row_stride, n + kRowStep, s.n1, rl, l, raw);
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       if (a.signs) hadamard_quad<D>(x[u], smask, lane, a.inv_sqrt_d);
@@ -249,44 +267,66 @@ __global__ void __launch_bounds__(kThreads) quant_qk_kernel(Args a) {
 
 // Pass 2b: V codes, transposed.  CTA = (b, h, 128-key block): 128 x D codes through shared
 // memory, written as D rows of up to 128 contiguous keys.  Keys in [N, Npad) are zero.
+// A work item is (4 consecutive keys, 8 consecutive head-dim elements): four 16-byte loads
+// (the lanes of a warp cover whole key rows, so the loads are coalesced), and per element one
+// 32-bit word holding its four keys' codes.  The tile holds words: row = head-dim element,
+// 32 words = 128 keys, and word w of row r sits at column w ^ (g * 32 / G) for element group
+// g = r / 8 (G groups per key), so that a warp's column writes (16 or 8 element groups x 2 or
+// 4 key quads) and its row reads both touch 32 different banks.
 template <int D>
 __global__ void __launch_bounds__(kThreads) quant_vt_kernel(Args a) {
-  __shared__ uint8_t tile[D][128 + 4];
+  constexpr int G = D / 8;                       // 8-element groups per key
+  constexpr int kItems = 32 * G / kThreads;      // work items per thread: 2 (d=128) or 1
+  constexpr int kSwz = 32 / G;                   // column XOR step per element group
+  __shared__ uint32_t tile[D][32];
   const int nblk = (a.npad + 127) / 128;
   const int blk = blockIdx.x % nblk;
   const int bh = blockIdx.x / nblk;
   const int b = bh / a.H, h = bh % a.H;
   const int n0 = blk * 128;
   const float inv = exp2i(-scale_exp(__uint_as_float(a.amax[2 * a.B * a.H + bh])));
-  // Load: thread handles (key, 8-element group); D/8 groups per key.
-  for (int i = threadIdx.x; i < 128 * (D / 8); i += kThreads) {
-    const int key = i / (D / 8), g = i % (D / 8);
-    const int n = n0 + key;
-    uint32_t c[4] = {0u, 0u, 0u, 0u};
-    if (n < a.N) {
-      const uint4 u = *reinterpret_cast<const uint4*>(
-          a.src_v + ((static_cast<size_t>(b) * a.N + n) * a.H + h) * D + g * 8);
-      c[0] = pack_e4m3x2(bf16_lo(u.x) * inv, bf16_hi(u.x) * inv);
-      c[1] = pack_e4m3x2(bf16_lo(u.y) * inv, bf16_hi(u.y) * inv);
-      c[2] = pack_e4m3x2(bf16_lo(u.z) * inv, bf16_hi(u.z) * inv);
-      c[3] = pack_e4m3x2(bf16_lo(u.w) * inv, bf16_hi(u.w) * inv);
-    }
+  const __nv_bfloat16* src = a.src_v + (static_cast<size_t>(b) * a.N * a.H + h) * D;
+  const size_t row_stride = static_cast<size_t>(a.H) * D;
+  uint4 u[kItems][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      tile[g * 8 + 2 * j][key] = static_cast<uint8_t>(c[j] & 0xFF);
-      tile[g * 8 + 2 * j + 1][key] = static_cast<uint8_t>(c[j] >> 8);
+  for (int it = 0; it < kItems; ++it) {
+    const int i = threadIdx.x + it * kThreads;
+    const int g = i % G, kq = i / G;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const int n = n0 + 4 * kq + kk;
+      u[it][kk] = n < a.N ? *reinterpret_cast<const uint4*>(src + n * row_stride + 8 * g)
+                          : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+#pragma unroll
+  for (int it = 0; it < kItems; ++it) {
+    const int i = threadIdx.x + it * kThreads;
+    const int g = i % G, kq = i / G;
+    const int col = kq ^ (g * kSwz);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {  // elements 8g + 2m, 8g + 2m + 1
+      uint32_t c[4];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t w = m == 0 ? u[it][kk].x : m == 1 ? u[it][kk].y : m == 2 ? u[it][kk].z : u[it][kk].w;
+        c[kk] = pack_e4m3x2(bf16_lo(w) * inv, bf16_hi(w) * inv);  // (element 2m, 2m + 1)
+      }
+      const uint32_t x = c[0] | (c[1] << 16), y = c[2] | (c[3] << 16);
+      tile[8 * g + 2 * m][col] = __byte_perm(x, y, 0x6420);      // keys 0..3, element 2m
+      tile[8 * g + 2 * m + 1][col] = __byte_perm(x, y, 0x7531);  // keys 0..3, element 2m + 1
     }
   }
   __syncthreads();
-  // Store: D rows x 128 keys, 4 bytes per thread.
+  // Store: D rows x 128 keys, one word (4 keys) per thread and row.
   const int nkeys = min(128, a.npad - n0);  // a multiple of 16
+  uint8_t* dst = a.vt + static_cast<size_t>(bh) * D * a.npad + n0;
+#pragma unroll
   for (int i = threadIdx.x; i < D * 32; i += kThreads) {
-    const int row = i / 32, q4 = i % 32;
-    if (q4 * 4 >= nkeys) continue;
-    const uint32_t v = tile[row][q4 * 4] | (tile[row][q4 * 4 + 1] << 8) |
-                       (tile[row][q4 * 4 + 2] << 16) | (static_cast<uint32_t>(tile[row][q4 * 4 + 3]) << 24);
-    *reinterpret_cast<uint32_t*>(a.vt + ((static_cast<size_t>(b) * a.H + h) * D + row) * a.npad +
-                                 n0 + q4 * 4) = v;
+    const int row = i / 32, w = i % 32;
+    if (4 * w >= nkeys) continue;
+    *reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(row) * a.npad + 4 * w) =
+        tile[row][w ^ ((row / 8) * kSwz)];
   }
 }
 
