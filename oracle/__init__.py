@@ -8,5 +8,6 @@ passage of the source pages each step follows.
 from .attention import (  # noqa: F401
     forward, backward, forward_head, backward_head,
     forward_rows, dq_rows, kv_grad_tail, scalar_loop_head, forward_head_block_sparse,
+    forward_rows_block_sparse,
 )
 from . import fp8  # noqa: F401,E402

@@ -257,3 +257,34 @@ def forward_head_block_sparse(Q, K, V, scale: float, causal: bool, block_mask, b
         P, lse[live] = _softmax_rows(S[live])
         O[live] = P @ V
     return O, lse
+
+
+def forward_rows_block_sparse(Q, K, V, scale: float, causal: bool, block_mask, rows,
+                              bq: int = 128, bk: int = 128) -> Tuple[np.ndarray, np.ndarray]:
+    """O [len(rows), d] and LSE [len(rows)] of the block-sparse attention above at the selected
+    query rows, without the N x N matrix (for long sequences): query i attends to the keys of
+    the active blocks of its block row (and, causal, j <= i), with the plain two-pass softmax
+    over that key set; a row with no such key gets O = 0, LSE = -inf."""
+    Q = np.asarray(Q, np.float64)
+    K = np.asarray(K, np.float64)
+    V = np.asarray(V, np.float64)
+    mask = np.asarray(block_mask).astype(bool)
+    nk = K.shape[0]
+    rows = np.asarray(rows)
+    O = np.zeros((len(rows), V.shape[1]))
+    lse = np.full(len(rows), -np.inf)
+    for n, i in enumerate(rows):
+        blocks = np.nonzero(mask[i // bq])[0]
+        if blocks.size == 0:
+            continue
+        keys = np.concatenate([np.arange(b * bk, min(nk, (b + 1) * bk)) for b in blocks])
+        if causal:
+            keys = keys[keys <= i]
+        if keys.size == 0:
+            continue
+        s = scale * (K[keys] @ Q[i])
+        m = s.max()
+        e = np.exp(s - m)
+        O[n] = (e @ V[keys]) / e.sum()
+        lse[n] = m + math.log(e.sum())
+    return O, lse

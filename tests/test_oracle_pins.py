@@ -364,3 +364,52 @@ def test_block_sparse_empty_rows_and_brute_force():
     # causal: block (0,1) lies above the diagonal, so rows 0..127 see nothing
     Oc, Lc = oracle.forward_head_block_sparse(Q, K, V, 0.5, True, m)
     assert np.all(Oc[:128] == 0) and np.all(np.isneginf(Lc[:128]))
+
+
+def test_block_sparse_rows_all_ones_equal_dense_rows():
+    # With every block active the sampled-rows form is dense attention at those rows.
+    N, d = 300, 8
+    Q, K, V = rnd(109, N, d), rnd(110, N, d), rnd(111, N, d)
+    rows = np.array([0, 1, 127, 128, 200, 299])
+    for causal in (False, True):
+        O, L = oracle.forward_rows_block_sparse(Q, K, V, 0.3, causal, np.ones((3, 3), np.uint8), rows)
+        Od, Ld = forward_head(Q, K, V, 0.3, causal)
+        np.testing.assert_allclose(O, Od[rows], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(L, Ld[rows], rtol=0, atol=1e-13)
+
+
+def test_block_sparse_rows_one_block_is_dense_attention_over_that_block():
+    # Block row r sees only key block p(r): its rows are non-causal dense attention over
+    # K, V rows [128 p, 128 p + 128) (the last block is ragged); block row 1 sees nothing.
+    N, d = 300, 8
+    Q, K, V = rnd(112, N, d), rnd(113, N, d), rnd(114, N, d)
+    m = np.zeros((3, 3), np.uint8)
+    m[0, 2] = 1
+    m[2, 0] = 1
+    rows = np.array([0, 50, 127, 128, 255, 256, 299])
+    O, L = oracle.forward_rows_block_sparse(Q, K, V, 0.7, False, m, rows)
+    for n, i in enumerate(rows):
+        if i // 128 == 1:
+            assert np.all(O[n] == 0) and np.isneginf(L[n])
+            continue
+        a = 256 if i // 128 == 0 else 0
+        Ob, Lb = forward_head(Q[i:i + 1], K[a:a + 128], V[a:a + 128], 0.7, False)
+        np.testing.assert_allclose(O[n], Ob[0], rtol=0, atol=1e-13)
+        assert abs(L[n] - Lb[0]) < 1e-12
+    # causal: block (0, 2) lies above the diagonal, so block row 0 sees nothing either
+    Oc, Lc = oracle.forward_rows_block_sparse(Q, K, V, 0.7, True, m, rows[:3])
+    assert np.all(Oc == 0) and np.all(np.isneginf(Lc))
+
+
+def test_block_sparse_rows_match_the_whole_head_form():
+    N, d = 390, 4
+    Q, K, V = rnd(115, N, d), rnd(116, N, d), rnd(117, N, d)
+    m = (np.random.default_rng(118).random((4, 4)) < 0.5).astype(np.uint8)
+    rows = np.arange(0, N, 7)
+    for causal in (False, True):
+        O, L = oracle.forward_rows_block_sparse(Q, K, V, 0.4, causal, m, rows)
+        Oh, Lh = oracle.forward_head_block_sparse(Q, K, V, 0.4, causal, m)
+        np.testing.assert_allclose(O, Oh[rows], rtol=0, atol=1e-13)
+        assert np.array_equal(np.isneginf(L), np.isneginf(Lh[rows]))
+        live = np.isfinite(L)
+        np.testing.assert_allclose(L[live], Lh[rows][live], rtol=0, atol=1e-12)
