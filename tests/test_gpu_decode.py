@@ -153,3 +153,53 @@ def test_block_sparse_interleaved_and_odd_tile_counts(fa, d, causal):
     m[3, :] = 0  # tile 3 sees nothing: O = 0, lse = -inf (its pair partner is tile 2)
     _bs_case(fa, 1, N, 3, d, causal, m, 6200 + d)
 
+
+
+def _bs_sampled(fa, B, N, H, d, causal, mask, seed, heads, rows):
+    """Block-sparse forward at full size, checked at sampled rows of a few heads."""
+    t = synthetic.draw(B, N, H, d, seed, "bf16")
+    q, k, v = (t[n].cuda() for n in ("q", "k", "v"))
+    scale = 1.0 / math.sqrt(d)
+    o, lse = fa.attention_block_sparse(q, k, v, torch.from_numpy(mask), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.fa_read_device_status() == 0
+    for b, h in heads:
+        Or, Lr = oracle.forward_rows_block_sparse(*(synthetic.to_f64(t[n][b, :, h]) for n in ("q", "k", "v")),
+                                                  scale, causal, mask, rows)
+        O, L = to_np(o[b, rows, h]), to_np(lse[b, h, rows])
+        live = np.isfinite(Lr)
+        assert np.all(np.isneginf(L[~live])) and np.all(O[~live] == 0)
+        assert max_abs(O, Or) <= O_MAX_ABS
+        assert rel_l2(O[live], Or[live]) <= O_REL_L2
+        assert max_abs(L[live], Lr[live]) <= LSE_MAX_ABS
+
+
+@pytest.mark.parametrize("d,causal", [(128, False), (128, True), (64, False)])
+def test_block_sparse_full_size_sampled_rows(fa, d, causal):
+    """The benchmark's block-sparse size (N = 16384, H*d = 2048, a random mask of density 0.5
+    with the diagonal kept): 128 query tiles per head, so each persistent CTA walks many units
+    with different active-tile counts; sampled rows of four heads."""
+    N, H = 16384, 2048 // d
+    nt = N // 128
+    m = (np.random.default_rng(400 + d).random((nt, nt)) < 0.5).astype(np.uint8)
+    m[np.arange(nt), np.arange(nt)] = 1
+    rng = np.random.default_rng(401 + d)
+    rows = np.unique(np.concatenate([[0, 127, 128, 255, 256, N - 129, N - 1], rng.integers(0, N, 41)]))
+    heads = [(0, 0), (0, H // 3), (0, H // 2), (0, H - 1)]
+    _bs_sampled(fa, 1, N, H, d, causal, m, 7000 + d, heads, rows)
+
+
+def test_block_sparse_longest_supported_sequence(fa):
+    """N = 131072, the documented limit (1024 key tiles: every one of a query tile's 32 bitmask
+    words is in use), with a causal band of 8 key tiles plus the first key tile, and a query
+    tile whose band is cut out; rows from the first, a middle and the last query tiles."""
+    N, H, d = 131072, 2, 128
+    nt = N // 128
+    m = np.zeros((nt, nt), np.uint8)
+    for i in range(nt):
+        m[i, max(0, i - 7):i + 1] = 1
+        m[i, 0] = 1
+    m[700, :] = 0  # this query tile sees nothing: O = 0, LSE = -inf
+    rows = np.array([0, 1, 127, 128, 700 * 128, 700 * 128 + 127, 701 * 128 + 5, 65535, 65536,
+                     N - 130, N - 129, N - 128, N - 2, N - 1])
+    _bs_sampled(fa, 1, N, H, d, True, m, 7100, [(0, 0), (0, 1)], rows)
